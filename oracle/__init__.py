@@ -1,0 +1,9 @@
+"""fp64 CPU oracle for exact attention (test infrastructure; see attention.py)."""
+from .attention import (  # noqa: F401
+    as_f64,
+    attention_bwd,
+    attention_fwd,
+    attention_fwd_blockwise,
+    attention_fwd_rows,
+    softmax_merge,
+)

@@ -1,0 +1,224 @@
+"""Plain fp64 CPU oracle for exact attention: forward, backward, softmax merge.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import this module:
+it is called by ``tests/``, by ``__graft_entry__.smoke()`` and by the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py``, and by nothing
+else.  It shares no code with the CUDA path (no kernels, headers, helpers or
+constants); both sides only share the seeded input generator, which holds none
+of the method's arithmetic.
+
+Sources (the pages this follows; cited by title and section):
+
+[P1] "Flash Attention: Rivoluzionando l'Efficienza dei Modelli Transformer"
+     (unite.ai): the ``standard_attention`` listing (definition of the result),
+     section "La Matematica dietro Flash Attention" (softmax decomposition and
+     the softmax merge), section "Dettagli di Implementazione" (the blockwise
+     algorithm with running statistics M, L).
+[P5] "Flash Attention: بهینه‌سازی مکانیزم توجه در ترنسفورمرها" (deepfa.ir):
+     section "ساختار مکانیزم توجه" (Attention(Q,K,V) = softmax(QK^T/sqrt d) V),
+     section "تکنیک 2: محاسبه مجدد" (the backward recomputes the attention
+     matrix instead of storing it).
+[P3] nearauto.com FlashAttention-2 digest, section on reducing non-matmul
+     FLOPs (normalise once, outputs unchanged).
+
+Every function here is the plain definition written out in float64 with numpy:
+the score matrix S and the probabilities P are materialised for whole rows,
+the softmax is two-pass (max, then exp / sum).  The only exception is
+``attention_fwd_blockwise``, which deliberately takes the pages' tiled steps so
+that the merge identity can be pinned against the two-pass definition.
+
+Readings where the pages are silent or garbled (each is listed in the design doc):
+  * layout [B, H, N, d]: the pages' (batch, seq, d) with a head axis added;
+  * lse is the natural log of sum_j exp(scale * q_i . k_j) over unmasked j;
+  * causal masks j > i (top-left aligned, N_q == N_k);
+  * the printed blockwise listing divides the output by the new running sum
+    while rescaling the old (already divided) output by exp(m_old - m_new)
+    alone; we keep the output unnormalised and divide once at the end;
+  * the garbled merge formula is read as l = e^(m_x-m) l_x + e^(m_y-m) l_y and
+    softmax(x u y) = [e^(m_x-m) l_x softmax(x), e^(m_y-m) l_y softmax(y)] / l;
+  * the backward is the exact gradient of the forward (the pages only say
+    "recompute"), with D_i = sum_j P_ij dP_ij.
+
+Parity pins for every function live in tests/test_oracle.py; none of the
+functions below is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "as_f64",
+    "attention_fwd",
+    "attention_fwd_rows",
+    "attention_bwd",
+    "softmax_merge",
+    "attention_fwd_blockwise",
+]
+
+
+def as_f64(x) -> np.ndarray:
+    """Return ``x`` as a C-contiguous float64 numpy array (exact for bf16/fp32)."""
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _scores(q_rows: np.ndarray, k: np.ndarray, scale: float, row_idx: np.ndarray,
+            causal: bool) -> np.ndarray:
+    """S = scale * Q K^T for the given query rows of one head, masked if causal.
+
+    [P1] ``standard_attention`` listing: scores = Q K^T / sqrt(d_k);
+    [P5] "ساختار مکانیزم توجه".  Causal: s_ij = -inf for j > i.
+    """
+    s = scale * (q_rows @ k.T)
+    if causal:
+        cols = np.arange(k.shape[0])
+        s = np.where(cols[None, :] > row_idx[:, None], -np.inf, s)
+    return s
+
+
+def _softmax_rows(s: np.ndarray):
+    """Two-pass safe softmax of complete rows; returns (P, lse).
+
+    [P1] "La Matematica dietro Flash Attention", softmax decomposition:
+    softmax(x) = exp(x - m) / sum exp(x - m) with m = max x.  The log-sum-exp
+    is m + ln(sum exp(x - m)).
+    """
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    denom = e.sum(axis=1, keepdims=True)
+    p = e / denom
+    lse = (m + np.log(denom))[:, 0]
+    return p, lse
+
+
+def attention_fwd(q, k, v, scale: float, causal: bool, panel_rows: int = 2048):
+    """O = softmax(scale Q K^T) V and lse per row, for [B, H, N, d] inputs.
+
+    [P1] ``standard_attention``; [P5] "ساختار مکانیزم توجه".  Materialises S
+    and P one head at a time, in panels of complete rows (each row is formed in
+    full before it is normalised), so memory stays bounded for long N.
+    The value width may differ from d (O takes V's last dimension).
+    Returns (O [B,H,N,d_v] float64, lse [B,H,N] float64).
+    """
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    B, H, N, d = q.shape
+    o = np.empty((B, H, N, v.shape[-1]), dtype=np.float64)
+    lse = np.empty((B, H, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, N, panel_rows):
+                rows = np.arange(r0, min(N, r0 + panel_rows))
+                s = _scores(q[b, h, rows], k[b, h], scale, rows, causal)
+                p, l_ = _softmax_rows(s)
+                o[b, h, rows] = p @ v[b, h]
+                lse[b, h, rows] = l_
+    return o, lse
+
+
+def attention_fwd_rows(q_rows, k, v, row_idx, scale: float, causal: bool):
+    """Forward for selected query rows of ONE head, against all N keys.
+
+    ``q_rows`` [R, d] are the query vectors of rows ``row_idx`` (their position
+    in the sequence, used by the causal mask); ``k``, ``v`` are [N, d].  Same
+    definition as ``attention_fwd``; used to check long sequences on sampled
+    rows.  Returns (O [R, d], lse [R]).
+    """
+    q_rows, k, v = as_f64(q_rows), as_f64(k), as_f64(v)
+    row_idx = np.asarray(row_idx, dtype=np.int64)
+    s = _scores(q_rows, k, scale, row_idx, causal)
+    p, lse = _softmax_rows(s)
+    return p @ v, lse
+
+
+def attention_bwd(q, k, v, do, scale: float, causal: bool):
+    """Exact gradients (dQ, dK, dV) of sum(dO * O) for O = attention_fwd(...).
+
+    [P5] "تکنیک 2: محاسبه مجدد": the backward recomputes P from Q, K (and the
+    saved statistics) instead of reading a stored N x N matrix.  The pages give
+    no formulas; the reading is the exact derivative of the forward:
+        dV = P^T dO,   dP = dO V^T,   D_i = sum_j P_ij dP_ij,
+        dS = P * (dP - D 1^T),   dQ = scale dS K,   dK = scale dS^T Q.
+    P is this oracle's own fp64 probability matrix (not a device result).
+    Returns float64 arrays shaped like q, k, v.
+    """
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    B, H, N, d = q.shape
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    rows = np.arange(N)
+    for b in range(B):
+        for h in range(H):
+            s = _scores(q[b, h], k[b, h], scale, rows, causal)
+            p, _ = _softmax_rows(s)
+            dv[b, h] = p.T @ do[b, h]
+            dp = do[b, h] @ v[b, h].T
+            dd = (p * dp).sum(axis=1, keepdims=True)
+            ds = p * (dp - dd)
+            dq[b, h] = scale * (ds @ k[b, h])
+            dk[b, h] = scale * (ds.T @ q[b, h])
+    return dq, dk, dv
+
+
+def softmax_merge(m_x, l_x, o_x, m_y, l_y, o_y):
+    """Merge two partial softmax-weighted results over disjoint key sets.
+
+    [P1] "La Matematica dietro Flash Attention", softmax merge, read as: with
+    m = max(m_x, m_y),  l = e^(m_x - m) l_x + e^(m_y - m) l_y, and the
+    normalised partial outputs o_x = sum_{j in x} softmax(x)_j v_j (likewise
+    o_y) combine into
+        o = (e^(m_x - m) l_x o_x + e^(m_y - m) l_y o_y) / l.
+    Arguments are per-row: m_*, l_* shaped [R], o_* shaped [R, d].  A row with
+    m = -inf on one side (no unmasked key there) takes the other side alone.
+    Returns (m, l, o).
+    """
+    m_x, l_x, o_x = as_f64(m_x), as_f64(l_x), as_f64(o_x)
+    m_y, l_y, o_y = as_f64(m_y), as_f64(l_y), as_f64(o_y)
+    m = np.maximum(m_x, m_y)
+    with np.errstate(invalid="ignore"):
+        a_x = np.where(np.isneginf(m_x), 0.0, np.exp(m_x - m))
+        a_y = np.where(np.isneginf(m_y), 0.0, np.exp(m_y - m))
+    w_x = a_x * l_x
+    w_y = a_y * l_y
+    l = w_x + w_y
+    o = (w_x[:, None] * o_x + w_y[:, None] * o_y) / l[:, None]
+    return m, l, o
+
+
+def attention_fwd_blockwise(q, k, v, scale: float, causal: bool,
+                            block_q: int = 64, block_k: int = 64):
+    """The pages' tiled forward with running row max M and row sum L.
+
+    [P1] "L'Algoritmo di Flash Attention" and "Dettagli di Implementazione":
+    queries in blocks, and for each query block a loop over key/value blocks
+    that updates M_new = max(M, rowmax S_block), L_new = e^(M - M_new) L +
+    rowsum e^(S_block - M_new), and the output.  Reading (see module doc): the
+    output is kept unnormalised, O <- e^(M - M_new) O + e^(S_block - M_new) V,
+    and divided by L once after the last key block ([P3], fewer non-matmul
+    FLOPs, same result).  Key blocks that are entirely masked are skipped.
+    Returns (O, lse) like ``attention_fwd``; equal to it up to rounding.
+    """
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    B, H, N, d = q.shape
+    o_out = np.empty_like(q)
+    lse_out = np.empty((B, H, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for i0 in range(0, N, block_q):
+                rows = np.arange(i0, min(N, i0 + block_q))
+                M = np.full(rows.size, -np.inf)
+                L = np.zeros(rows.size)
+                O = np.zeros((rows.size, d))
+                for j0 in range(0, N, block_k):
+                    if causal and j0 > rows[-1]:
+                        break
+                    cols = slice(j0, min(N, j0 + block_k))
+                    s = _scores(q[b, h, rows], k[b, h, cols], scale,
+                                rows - j0, causal)
+                    m_new = np.maximum(M, s.max(axis=1))
+                    p = np.exp(s - m_new[:, None])
+                    with np.errstate(invalid="ignore"):
+                        alpha = np.where(np.isneginf(M), 0.0, np.exp(M - m_new))
+                    L = alpha * L + p.sum(axis=1)
+                    O = alpha[:, None] * O + p @ v[b, h, cols]
+                    M = m_new
+                o_out[b, h, rows] = O / L[:, None]
+                lse_out[b, h, rows] = M + np.log(L)
+    return o_out, lse_out
