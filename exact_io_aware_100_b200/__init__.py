@@ -1,0 +1,173 @@
+"""Python binding of libfa.so (exact IO-aware attention for B200, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/fa.h``.  PyTorch provides device
+memory and streams.  There is no CPU fallback: if ``libfa.so`` is missing the
+calls raise.
+
+Low-level names mirror the C ABI (``fa_fwd``, ``fa_fwd_ex``, ``fa_bwd``, ...)
+and take torch tensors for the pointer arguments.  ``forward`` / ``backward``
+allocate the outputs (and workspace) with torch and call them.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_ALIGN, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(7)
+FA_BF16, FA_F32 = 0, 1
+
+EXPORTS = (
+    "fa_fwd", "fa_fwd_ex", "fa_fwd_workspace_size", "fa_bwd", "fa_bwd_workspace_size",
+    "fa_get_device_status", "fa_selftest_wait_timeout", "fa_status_string", "fa_version",
+)
+
+
+class FaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where} failed: {status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfa.so and declare the C signatures (no GPU needed)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built; run `python -m exact_io_aware_100_b200.build`")
+    L = ctypes.CDLL(path)
+    P, I, F, Z, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+    L.fa_fwd.argtypes = [P, P, P, P, P, I, I, I, I, F, I, P]
+    L.fa_fwd_ex.argtypes = [P, P, P, P, P, I, I, I, I, F, I, I, P, Z, P]
+    L.fa_fwd_workspace_size.argtypes = [I, I, I, I, I]
+    L.fa_fwd_workspace_size.restype = Z
+    L.fa_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, Z, P]
+    L.fa_bwd_workspace_size.argtypes = [I, I, I, I]
+    L.fa_bwd_workspace_size.restype = Z
+    L.fa_get_device_status.argtypes = [P]
+    L.fa_selftest_wait_timeout.argtypes = [U64, P]
+    L.fa_status_string.argtypes = [I]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_version.restype = ctypes.c_char_p
+    for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_get_device_status", "fa_selftest_wait_timeout"):
+        getattr(L, name).restype = I
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return load_library().fa_status_string(int(code)).decode()
+
+
+def version() -> str:
+    return load_library().fa_version().decode()
+
+
+def _check(code: int, where: str) -> None:
+    if code != FA_OK:
+        raise FaError(code, where)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _bhnd(t):
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError("expected a contiguous [B, H, N, d] tensor")
+    return t.shape
+
+
+# ----------------------------------------------------------------- C ABI mirrors
+def fa_fwd(q, k, v, o, lse, causal: bool, scale: float | None = None, stream=None) -> None:
+    B, H, N, d = _bhnd(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(load_library().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
+                                 int(bool(causal)), _stream(stream)), "fa_fwd")
+
+
+def fa_fwd_ex(q, k, v, o, lse, causal: bool, dtype: int, workspace, scale: float | None = None,
+              stream=None) -> None:
+    B, H, N, d = _bhnd(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, scale,
+                                    int(bool(causal)), int(dtype), _ptr(workspace), ws_bytes,
+                                    _stream(stream)), "fa_fwd_ex")
+
+
+def fa_fwd_workspace_size(B: int, H: int, N: int, d: int, dtype: int) -> int:
+    return int(load_library().fa_fwd_workspace_size(B, H, N, d, dtype))
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, workspace, scale: float | None = None,
+           stream=None) -> None:
+    B, H, N, d = _bhnd(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                                 _ptr(dk), _ptr(dv), B, H, N, d, scale, int(bool(causal)),
+                                 _ptr(workspace), ws_bytes, _stream(stream)), "fa_bwd")
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().fa_bwd_workspace_size(B, H, N, d))
+
+
+def fa_get_device_status(stream=None) -> int:
+    return int(load_library().fa_get_device_status(_stream(stream)))
+
+
+def fa_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:
+    _check(load_library().fa_selftest_wait_timeout(int(timeout_ns), _stream(stream)),
+           "fa_selftest_wait_timeout")
+
+
+# ----------------------------------------------------------------- conveniences
+def _workspace(nbytes: int, device):
+    import torch
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def forward(q, k, v, causal: bool, scale: float | None = None, stream=None):
+    """O, lse for [B,H,N,d] tensors (bf16, or float32 via the bf16 tensor-core path)."""
+    import torch
+    B, H, N, d = _bhnd(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if q.dtype == torch.bfloat16:
+        fa_fwd(q, k, v, o, lse, causal, scale, stream)
+    elif q.dtype == torch.float32:
+        ws = _workspace(fa_fwd_workspace_size(B, H, N, d, FA_F32), q.device)
+        fa_fwd_ex(q, k, v, o, lse, causal, FA_F32, ws, scale, stream)
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    return o, lse
+
+
+def backward(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, stream=None, workspace=None):
+    """dQ, dK, dV (bf16) from the forward's O and lse."""
+    import torch
+    B, H, N, d = _bhnd(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = _workspace(fa_bwd_workspace_size(B, H, N, d), q.device)
+    fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal, workspace, scale, stream)
+    return dq, dk, dv

@@ -1,0 +1,402 @@
+// Forward attention kernel for sm_100a: O = softmax(scale Q K^T) V, lse per row.
+//
+// The method (exact attention computed tile by tile with the online-softmax
+// rescaling, so the N x N score matrix never leaves the chip) is the one the
+// unite.ai page "Flash Attention: Rivoluzionando l'Efficienza dei Modelli
+// Transformer" describes in "L'Algoritmo di Flash Attention" and "La Matematica
+// dietro Flash Attention" (softmax decomposition and merge); the deferred
+// normalisation and the skipping of fully masked causal tiles follow the
+// nearauto.com FlashAttention-2 digest ("reducing non-matmul FLOPs", "better
+// parallelism": query-row blocks spread over all SMs, sequence dimension too).
+//
+// B200 design (not the pages' A100 / H100 partitioning):
+//  * persistent CTAs, one per SM, walk work tiles of 256 query rows of one
+//    (batch, head); causal tiles are visited longest first;
+//  * warp roles: warps 0-3 and 4-7 are two softmax warpgroups, each owning one
+//    128-row half of the tile (thread t owns TMEM lane / query row t); warp 8
+//    issues the tcgen05 MMAs from one thread; warp 9 issues TMA loads from one
+//    thread; warps 10-11 only take part in set-up and teardown;
+//  * TMA streams K_j and V_j (128 keys each) through a ring of shared-memory
+//    stages with full / empty mbarriers; Q (both halves) is loaded once per tile;
+//  * tensor memory (512 columns): S0 | S1 | O0 | O1; P (bf16) is written back
+//    over the first half of its S columns and fed to the P.V MMA from TMEM;
+//  * MMA issue order per KV block j: S0_j, P1V_{j-1}, S1_j, P0V_j, so one
+//    half's softmax overlaps the other half's MMAs (ping-pong);
+//  * the softmax keeps a per-row reference max m and sum l; it rescales O in
+//    TMEM only when the block max exceeds m by more than 2^8 in exp2 units
+//    (exact: the final O / l uses the same reference), warp-uniformly;
+//  * every mbarrier wait is bounded; on timeout the CTA sets the status word,
+//    drains its own in-flight copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fa {
+
+struct FwdArgs {
+  void* o;              // [BH, N, D] bf16 or f32
+  float* lse;           // [BH, N] natural-log logsumexp
+  uint32_t* status;     // device status word
+  int N;
+  int bh;               // B * H
+  int n_qt;             // ceil(N / 256)
+  int n_kv_all;         // ceil(N / 128)
+  int num_tiles;        // bh * n_qt
+  int causal;
+  int o_f32;
+  float scale_log2;     // scale * log2(e)
+  unsigned long long wait_limit_ns;
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128;                  // query rows per softmax warpgroup
+  static constexpr int BN = 128;                  // keys per KV block
+  static constexpr int TILE_M = 2 * BM;           // query rows per work tile
+  static constexpr int REGION = 128 * 128;        // one 64-column (128 B) swizzle region of a 128-row tile
+  static constexpr int N_REG = D / 64;            // regions per 128-row tile
+  static constexpr int Q_HALF = BM * D * 2;       // bytes of one 128-row Q half
+  static constexpr int KV_BYTES = BN * D * 2;     // bytes of one K or V block
+  static constexpr int STAGES = (D == 128) ? 4 : 8;
+  static constexpr int THREADS = 384;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
+  // shared-memory layout (offsets from a 1024-aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = 2 * Q_HALF;
+  static constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
+  // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, drain
+  static constexpr int N_BARS = 2 + 2 * STAGES + 2 + 2 + 2;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;   // tmem slot, abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024; // + alignment slack
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
+};
+
+__device__ __forceinline__ void fwd_decode_tile(const FwdArgs& a, int t, int& bh, int& qt) {
+  if (a.causal) {            // longest work first
+    qt = a.n_qt - 1 - t / a.bh;
+    bh = t % a.bh;
+  } else {                   // neighbouring CTAs share a head's K / V in L2
+    bh = t / a.n_qt;
+    qt = t % a.n_qt;
+  }
+}
+
+__device__ __forceinline__ int fwd_num_kv(const FwdArgs& a, int qt) {
+  if (!a.causal) return a.n_kv_all;
+  const int last_row = min(qt * 256 + 255, a.N - 1);
+  return last_row / 128 + 1;
+}
+
+template <int D>
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::OFF_Q;
+  const uint32_t sKV = sbase + C::OFF_KV;
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const uint32_t b_q_full = bar0, b_q_empty = bar0 + 8;
+  auto b_kv_full = [&](int s) { return bar0 + 16 + 8 * s; };
+  auto b_kv_empty = [&](int s) { return bar0 + 16 + 8 * C::STAGES + 8 * s; };
+  const uint32_t b_s_full0 = bar0 + 16 + 16 * C::STAGES;
+  const uint32_t b_p_full0 = b_s_full0 + 16;
+  const uint32_t b_o_done = b_p_full0 + 16;
+  const uint32_t b_drain = b_o_done + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0u;
+    mbar_init(b_q_full, 1);
+    mbar_init(b_q_empty, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(b_kv_full(s), 1);
+      mbar_init(b_kv_empty(s), 1);
+    }
+    mbar_init(b_s_full0, 1);
+    mbar_init(b_s_full0 + 8, 1);
+    mbar_init(b_p_full0, 128);
+    mbar_init(b_p_full0 + 8, 128);
+    mbar_init(b_o_done, 1);
+    mbar_init(b_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 8) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  if (warp == 9 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl ctl{abort_flag, args.status, args.wait_limit_ns};
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t kv_it = 0, tile_cnt = 0;
+      bool ok = true, q_pending = false;
+      uint32_t q_parity = 0;
+      uint32_t issued = 0, last_parity = 0;      // per-stage bit masks
+      for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x, ++tile_cnt) {
+        int bh, qt;
+        fwd_decode_tile(args, t, bh, qt);
+        const int nkv = fwd_num_kv(args, qt);
+        if (tile_cnt > 0 && !mbar_wait(b_q_empty, (tile_cnt - 1) & 1, ctl)) { ok = false; break; }
+        mbar_expect_tx(b_q_full, 2 * C::Q_HALF);
+        for (int h = 0; h < 2; ++h)
+          for (int r = 0; r < C::N_REG; ++r)
+            tma_load_3d(sQ + h * C::Q_HALF + r * C::REGION, &tm_q, b_q_full, r * 64, qt * 256 + h * 128, bh);
+        q_pending = true;
+        q_parity = tile_cnt & 1;
+        for (int j = 0; j < nkv && ok; ++j) {
+          for (int kind = 0; kind < 2; ++kind, ++kv_it) {
+            const int s = kv_it % C::STAGES;
+            const uint32_t round = kv_it / C::STAGES;
+            if (round > 0 && !mbar_wait(b_kv_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
+            mbar_expect_tx(b_kv_full(s), C::KV_BYTES);
+            const CUtensorMap* map = kind ? &tm_v : &tm_k;
+            for (int r = 0; r < C::N_REG; ++r)
+              tma_load_3d(sKV + s * C::KV_BYTES + r * C::REGION, map, b_kv_full(s), r * 64, j * 128, bh);
+            issued |= 1u << s;
+            last_parity = (last_parity & ~(1u << s)) | ((round & 1u) << s);
+          }
+        }
+      }
+      if (!ok) {   // drain our own copies still in flight before the CTA exits
+        for (int s = 0; s < C::STAGES; ++s)
+          if ((issued >> s) & 1u) mbar_wait_quiet(b_kv_full(s), (last_parity >> s) & 1u, 200000000ull);
+        if (q_pending) mbar_wait_quiet(b_q_full, q_parity, 200000000ull);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t kv_it = 0, tile_cnt = 0, p_par0 = 0, p_par1 = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x, ++tile_cnt) {
+        int bh, qt;
+        fwd_decode_tile(args, t, bh, qt);
+        const int nkv = fwd_num_kv(args, qt);
+        if (!mbar_wait(b_q_full, tile_cnt & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+        int sv_prev = 0;
+        for (int j = 0; j < nkv; ++j) {
+          // ---- K_j: S0 = Q0 K^T
+          const int sk = kv_it % C::STAGES;
+          if (!mbar_wait(b_kv_full(sk), (kv_it / C::STAGES) & 1, ctl)) { ok = false; break; }
+          ++kv_it;
+          tc_fence_after();
+          const uint32_t kbase = sKV + sk * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::REGION + (kk & 3) * 32;
+            umma_ss(tmem + C::T_S0, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
+                    C::IDESC_S, kk > 0);
+          }
+          umma_commit(b_s_full0);
+          // ---- O1 += P1 V_{j-1}
+          if (j > 0) {
+            if (!mbar_wait(b_p_full0 + 8, p_par1, ctl)) { ok = false; break; }
+            p_par1 ^= 1;
+            tc_fence_after();
+            const uint32_t vbase = sKV + sv_prev * C::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < C::BN / 16; ++kk)
+              umma_ts(tmem + C::T_O1, tmem + C::T_S1 + kk * 8, sdesc_sw128(vbase + kk * 2048, C::REGION, 1024),
+                      C::IDESC_PV, (j > 1) || (kk > 0));
+            umma_commit(b_kv_empty(sv_prev));
+          }
+          // ---- S1 = Q1 K^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::REGION + (kk & 3) * 32;
+            umma_ss(tmem + C::T_S1, sdesc_sw128(sQ + C::Q_HALF + off, 16, 1024),
+                    sdesc_sw128(kbase + off, 16, 1024), C::IDESC_S, kk > 0);
+          }
+          umma_commit(b_s_full0 + 8);
+          umma_commit(b_kv_empty(sk));
+          if (j == nkv - 1) umma_commit(b_q_empty);
+          // ---- V_j: O0 += P0 V_j
+          const int sv = kv_it % C::STAGES;
+          if (!mbar_wait(b_kv_full(sv), (kv_it / C::STAGES) & 1, ctl)) { ok = false; break; }
+          ++kv_it;
+          if (!mbar_wait(b_p_full0, p_par0, ctl)) { ok = false; break; }
+          p_par0 ^= 1;
+          tc_fence_after();
+          const uint32_t vbase = sKV + sv * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk)
+            umma_ts(tmem + C::T_O0, tmem + C::T_S0 + kk * 8, sdesc_sw128(vbase + kk * 2048, C::REGION, 1024),
+                    C::IDESC_PV, (j > 0) || (kk > 0));
+          sv_prev = sv;
+        }
+        if (!ok) break;
+        // ---- O1 += P1 V_last
+        if (!mbar_wait(b_p_full0 + 8, p_par1, ctl)) { ok = false; break; }
+        p_par1 ^= 1;
+        tc_fence_after();
+        {
+          const uint32_t vbase = sKV + sv_prev * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk)
+            umma_ts(tmem + C::T_O1, tmem + C::T_S1 + kk * 8, sdesc_sw128(vbase + kk * 2048, C::REGION, 1024),
+                    C::IDESC_PV, (nkv > 1) || (kk > 0));
+        }
+        umma_commit(b_kv_empty(sv_prev));
+        umma_commit(b_o_done);
+      }
+      // every MMA issued by this thread has completed before TMEM is freed
+      umma_commit(b_drain);
+      mbar_wait_quiet(b_drain, 0, 200000000ull);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int half = warp >> 2;                       // which 128-row half
+    const int rloc = (warp & 3) * 32 + lane;          // TMEM lane == row within the half
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (half ? C::T_S1 : C::T_S0);
+    const uint32_t tO = tmem + lane_off + (half ? C::T_O1 : C::T_O0);
+    const uint32_t b_s_full = b_s_full0 + 8 * half;
+    const uint32_t b_p_full = b_p_full0 + 8 * half;
+    const float c2 = args.scale_log2;
+    uint32_t s_par = 0, tile_cnt = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x, ++tile_cnt) {
+      int bh, qt;
+      fwd_decode_tile(args, t, bh, qt);
+      const int nkv = fwd_num_kv(args, qt);
+      const int row0 = qt * 256 + half * 128;
+      const int row = row0 + rloc;
+      const int lim = args.causal ? min(row + 1, args.N) : args.N;         // keys < lim are visible
+      const int lim_min = args.causal ? min(row0 + 1, args.N) : args.N;    // smallest lim in the warpgroup
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkv; ++j) {
+        if (!mbar_wait_warp(b_s_full, s_par, ctl)) { ok = false; break; }
+        s_par ^= 1;
+        tc_fence_after();
+        uint32_t sr[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+        const int kv0 = j * 128;
+        if (kv0 + 128 > lim_min) {          // diagonal or tail block: mask keys >= lim
+          const int cut = lim - kv0;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= cut) s[c] = -INFINITY;
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float m_new = fmaxf(m_ref, mx);
+        const bool need = (m_new - m_ref) * c2 > 8.0f;
+        const bool rescale = __any_sync(0xffffffffu, need);   // warp-uniform decision
+        float alpha = 1.0f;
+        if (rescale) {
+          alpha = ex2_approx((m_ref - m_new) * c2);              // 0 on the first block
+          l *= alpha;
+          m_ref = m_new;
+        }
+        const float negm = -m_ref * c2;
+        float l0 = 0.f, l1 = 0.f;
+        uint32_t pr[64];
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float p0 = ex2_approx(fmaf(s[c], c2, negm));
+          const float p1 = ex2_approx(fmaf(s[c + 1], c2, negm));
+          l0 += p0;
+          l1 += p1;
+          pr[c >> 1] = pack_bf16x2(p0, p1);
+        }
+        l += l0 + l1;
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pr));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pr + 32));
+        // O rescale (after the scores are dead, to keep register pressure down).
+        // Safe: S_j's commit covered every earlier MMA, including P V_{j-1} into O.
+        if (rescale && j > 0) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+            reg_fence32(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + c * 32, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(b_p_full);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> global, lse
+      if (!mbar_wait_warp(b_o_done, tile_cnt & 1, ctl)) { ok = false; break; }
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const bool valid = row < args.N;
+      const size_t grow = static_cast<size_t>(bh) * args.N + row;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+        if (valid) {
+          if (args.o_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.o) + grow * D + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
+                                   __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.o) + grow * D + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv_l, __uint_as_float(o[8 * e + 1]) * inv_l);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv_l, __uint_as_float(o[8 * e + 3]) * inv_l);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv_l, __uint_as_float(o[8 * e + 5]) * inv_l);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv_l, __uint_as_float(o[8 * e + 7]) * inv_l);
+              dst[e] = w;
+            }
+          }
+        }
+      }
+      if (valid) args.lse[grow] = (m_ref * c2 + __log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,124 @@
+/*
+ * fa.h -- C ABI of the exact IO-aware attention library (libfa.so, sm_100a).
+ *
+ * What is computed (exact attention, no approximation):
+ *     S = scale * Q K^T,  P = softmax_rows(S),  O = P V,
+ *     lse_i = ln sum_j exp(S_ij)  (natural log, over unmasked j).
+ * Definition: unite.ai, "Flash Attention: Rivoluzionando l'Efficienza dei
+ * Modelli Transformer", the standard_attention listing; deepfa.ir, "Flash
+ * Attention: بهینه‌سازی مکانیزم توجه در ترنسفورمرها", section on the
+ * attention structure.  It is computed tile by tile with the online-softmax
+ * rescaling of "La Matematica dietro Flash Attention" (softmax decomposition
+ * and merge), so the N x N matrix never reaches device memory.  The backward
+ * recomputes P from Q, K and lse (deepfa.ir, section "Technique 2:
+ * recomputation") and returns the exact gradients
+ *     dV = P^T dO,  dS = P * (dO V^T - D),  D_i = sum_c dO_ic O_ic,
+ *     dQ = scale dS K,  dK = scale dS^T Q.
+ * Causal masking hides key j from query i when j > i (top-left aligned,
+ * equal query and key lengths).
+ *
+ * Conventions shared by every call:
+ *  - Layout: q, k, v, o, dO, dq, dk, dv are dense row-major [B, H, N, d] with d
+ *    innermost (element strides d, N*d, H*N*d).  lse is dense [B, H, N] float.
+ *  - All pointers are DEVICE pointers owned by the caller; the library keeps
+ *    no reference after the call returns and allocates nothing on these paths.
+ *    Every pointer must be non-null and 16-byte aligned.
+ *  - Work is enqueued asynchronously on `stream` (0 = legacy default stream);
+ *    the functions never synchronise.  Argument errors are reported before
+ *    anything is launched.  A kernel whose internal wait gives up (a bug, or a
+ *    device that stopped making progress) sets a device status word that
+ *    fa_get_device_status() reports; outputs are then undefined.
+ *  - Supported: d in {64, 128} for the forward, d == 128 for the backward;
+ *    1 <= N <= 2^24; B*H*N*d < 2^31 elements per tensor.
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID = 1,      /* bad sizes (B, H, N < 1, N too large, non-finite scale) */
+  FA_ERR_UNSUPPORTED = 2,  /* d or dtype not supported by this call                 */
+  FA_ERR_ALIGN = 3,        /* null or not 16-byte aligned pointer                     */
+  FA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required              */
+  FA_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed                    */
+  FA_ERR_TIMEOUT = 6       /* a kernel's bounded internal wait gave up                */
+} fa_status;
+
+typedef enum {
+  FA_BF16 = 0,             /* bfloat16 q, k, v and o                                  */
+  FA_F32 = 1               /* float32 q, k, v and o (computed on the bf16 path)       */
+} fa_dtype;
+
+/* Opaque CUDA stream handle (a cudaStream_t). */
+typedef void* fa_stream_t;
+
+/*
+ * Forward, bf16.  q, k, v: [B,H,N,d] bf16 (read); o: [B,H,N,d] bf16 (written);
+ * lse: [B,H,N] float (written).  scale multiplies the scores (1/sqrt(d) for the
+ * usual attention).  causal != 0 applies the mask j > i.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, float scale, int causal, fa_stream_t stream);
+
+/*
+ * Forward with an element type.  FA_BF16 behaves like fa_fwd (workspace may be
+ * null).  FA_F32: q, k, v, o are float32; q, k, v are first rounded to bf16
+ * (nearest-even) into the caller's workspace, the product runs on the bf16
+ * tensor-core path with fp32 accumulation, and o is written as float32.
+ * workspace: device memory of at least fa_fwd_workspace_size(...) bytes,
+ * 256-byte aligned.
+ */
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int H, int N, int d, float scale, int causal, fa_dtype dtype,
+                    void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/* Bytes of workspace fa_fwd_ex needs (0 for FA_BF16). */
+size_t fa_fwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype);
+
+/*
+ * Backward, bf16, d == 128.  Inputs q, k, v, o, dO: [B,H,N,d] bf16; lse from the
+ * forward: [B,H,N] float.  Outputs dq, dk, dv: [B,H,N,d] bf16 (written, not
+ * accumulated).  workspace: device memory of at least fa_bwd_workspace_size()
+ * bytes, 256-byte aligned (holds the fp32 dQ accumulator and per-row D, lse).
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv,
+                 int B, int H, int N, int d, float scale, int causal,
+                 void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/* Bytes of workspace fa_bwd needs. */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device.  Returns FA_ERR_TIMEOUT if any kernel since the last call
+ * gave up a bounded wait, FA_ERR_CUDA if the synchronisation failed, else FA_OK.
+ */
+fa_status fa_get_device_status(fa_stream_t stream);
+
+/*
+ * Diagnostic: launches one tiny kernel that waits on a shared-memory barrier
+ * nothing will ever complete, bounded by timeout_ns (clamped to [1 ms, 2 s]).
+ * The kernel gives up, sets the status word and returns; the caller then sees
+ * FA_ERR_TIMEOUT from fa_get_device_status().  Used to test that path.
+ */
+fa_status fa_selftest_wait_timeout(uint64_t timeout_ns, fa_stream_t stream);
+
+/* Human-readable name of a status code. */
+const char* fa_status_string(fa_status s);
+
+/* Library version, e.g. "0.1.0". */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */
