@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Benchmark: exact attention forward + backward TFLOP/s on B200.
+
+One step = one pass of the whole path over one batch: the forward kernel
+(O, lse) and the three backward phases (prepare, main, finish).  Default
+workload: B=2 H=32 N=8192 d=128 bf16, K scaled by 2, causal (the prefill-shaped
+configuration the >=60%-of-peak target names).  FLOPs follow the pages'
+convention: forward 4*B*H*N^2*d (halved for causal), backward 2.5x forward.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...     # the fp64 CPU oracle on the same workload
+
+Under torchrun each rank runs the same per-GPU workload on its own seeded
+batch (weak scaling, no data-path collective); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from exact_io_aware_100_b200 import inputs  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOP/s (bf16, causal & non-causal); % of B200 BF16 peak"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["exact_io_aware_100_b200/csrc/ptx.cuh", "exact_io_aware_100_b200/csrc/fwd_kernel.cuh",
+                  "exact_io_aware_100_b200/csrc/bwd_kernel.cuh"]
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="prefill", choices=sorted(inputs.WORKLOADS))
+    p.add_argument("--fwd-only", action="store_true", help="time the forward kernel alone")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-heads", type=int, default=2, help="heads in the CPU baseline sample")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still matches the source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get("kernels", {}).get(kernel)
+    if not e or e.get("csrc_sha256") != kernel_source_hash() or e.get("workload") != workload:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML during the timed region."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:   # NVML unavailable: report nothing rather than guess
+            self.nv = None
+
+    def _handle(self, idx):
+        """NVML handle of CUDA device `idx`: match UUIDs, else CUDA_VISIBLE_DEVICES, else idx."""
+        import torch
+        pynvml = self.nv
+        try:
+            want = "GPU-" + str(torch.cuda.get_device_properties(idx).uuid)
+            for j in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(j)
+                got = pynvml.nvmlDeviceGetUUID(h)
+                got = got.decode() if isinstance(got, bytes) else str(got)
+                if got == want:
+                    return h
+        except Exception:
+            pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        parts = [p.strip() for p in vis.split(",") if p.strip()]
+        if idx < len(parts) and parts[idx].isdigit():
+            return pynvml.nvmlDeviceGetHandleByIndex(int(parts[idx]))
+        return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _reasons(self):
+        f = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return f(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self._reasons()
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, heads: int, seed_offset: int = 0, fwd_only: bool = False):
+    """fwd (+ bwd) of `heads` whole heads of the workload with the fp64 oracle.
+    Returns (seconds, algorithmic FLOPs of the sample, description)."""
+    from oracle import attention_bwd, attention_fwd
+    shape1 = (1, 1, w.N, w.d)
+    t_total, flops = 0.0, 0.0
+    for i in range(heads):
+        seed = w.seed + 7919 * (i + 1 + seed_offset)
+        f = {n: inputs.to_f64(inputs.make_tensor(seed, n, shape1, w.k_scale if n == "k" else 1.0), "bf16")
+             for n in ("q", "k", "v", "do")}
+        t0 = time.perf_counter()
+        attention_fwd(f["q"], f["k"], f["v"], w.scale, w.causal)
+        if not fwd_only:
+            attention_bwd(f["q"], f["k"], f["v"], f["do"], w.scale, w.causal)
+        t_total += time.perf_counter() - t0
+        flops += (1.0 if fwd_only else 3.5) * 4.0 * w.N * w.N * w.d / (2 if w.causal else 1)
+    desc = (f"{'fwd' if fwd_only else 'fwd+bwd'} of {heads} whole head(s) (1 x 1 x {w.N} x {w.d}) "
+            f"of the workload, numpy float64 oracle")
+    return t_total, flops, desc
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    fwd_only = is_fwd_only(args, w)
+    for _ in range(args.warmup):
+        oracle_sample(w, 1, seed_offset=1000, fwd_only=fwd_only)
+    secs, flops = 0.0, 0.0
+    for s in range(args.steps):
+        t, f, desc = oracle_sample(w, 1, seed_offset=s, fwd_only=fwd_only)
+        secs += t
+        flops += f
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, "fwd" if fwd_only else "fwd+bwd",
+                                  "oracle on host cores; each step one whole head"),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def is_fwd_only(args, w) -> bool:
+    """The backward kernel covers d = 128 with bf16 inputs; other workloads time the forward."""
+    return args.fwd_only or w.d != 128 or w.dtype != "bf16"
+
+
+def workload_config(w, step: str, note: str):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} {'causal' if w.causal else 'non-causal'}"
+                        + (f" K*{w.k_scale:g}" if w.k_scale != 1.0 else ""),
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "step": step, "l2": note}
+
+
+# --------------------------------------------------------------------- GPU arm
+def main():
+    args = parse_args()
+    w = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+    import torch
+    import torch.distributed as dist
+    import exact_io_aware_100_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    fa.load_library()
+
+    fwd_only = is_fwd_only(args, w)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    shape = (B, H, N, d)
+    seed = w.seed + 100003 * rank          # each rank its own batch
+    names = ("q", "k", "v") if fwd_only else ("q", "k", "v", "do")
+    host = {n: inputs.make_tensor(seed, n, shape, w.k_scale if n == "k" else 1.0, "bf16") for n in names}
+    pinned = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in names}
+    dv_ = {n: pinned[n].to(dev) for n in names}
+    o = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    if not fwd_only:
+        dq, dk, dvv = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
+        ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    causal = w.causal
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fa.fa_fwd(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if fwd_only:
+            return
+        fa.fa_bwd_prepare(o, lse, dv_["do"], ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        fa.fa_bwd_main(dv_["q"], dv_["k"], dv_["v"], dv_["do"], dk, dvv, causal, ws, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        fa.fa_bwd_finish(dq, ws, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    launches_per_step = 1 if fwd_only else 4
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_get_device_status() != fa.FA_OK:
+        raise SystemExit("device status reported a timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    if fa.fa_get_device_status() != fa.FA_OK:
+        raise SystemExit("device status reported a timeout in the timed region")
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    main_ms = None if fwd_only else statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    prep_ms = None if fwd_only else statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    fin_ms = None if fwd_only else statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    fwd_flops = w.fwd_flops()
+    bwd_flops = 2.5 * fwd_flops
+    step_flops = fwd_flops + (0.0 if fwd_only else bwd_flops)
+    value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+
+    fwd_tf = fwd_flops / (fwd_ms * 1e-3) / 1e12
+    kernels = {"fa_fwd_kernel": {"ms": fwd_ms, "tflops": fwd_tf, "frac_of_measured_burst": fwd_tf / burst,
+                                 "frac_of_datasheet": fwd_tf / DATASHEET_BF16_TFLOPS}}
+    if not fwd_only:
+        main_tf = bwd_flops / (main_ms * 1e-3) / 1e12
+        kernels["fa_bwd_kernel"] = {"ms": main_ms, "tflops": main_tf, "frac_of_measured_burst": main_tf / burst,
+                                    "frac_of_datasheet": main_tf / DATASHEET_BF16_TFLOPS}
+        kernels["fa_bwd_pre_kernel"] = {"ms": prep_ms}
+        kernels["fa_bwd_dq_kernel"] = {"ms": fin_ms}
+    dom = "fa_fwd_kernel" if (fwd_only or fwd_ms >= main_ms) else "fa_bwd_kernel"
+    dom_flops = fwd_flops if dom == "fa_fwd_kernel" else bwd_flops
+    achieved = kernels[dom]["tflops"]
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                "frac": achieved / burst, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "flops_per_launch": dom_flops, "traffic": committed_traffic(dom, w.name)}
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        outs = {"o": o, "lse": lse} if fwd_only else {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dvv}
+        host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in outs.items()}
+        h2d = sum(pinned[n].numel() * pinned[n].element_size() for n in names)
+        d2h = sum(t.numel() * t.element_size() for t in outs.values())
+
+        def e2e_step():
+            for n in names:
+                dv_[n].copy_(pinned[n], non_blocking=True)
+            step()
+            for n, t in outs.items():
+                host_out[n].copy_(t, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * step_flops * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms / args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, flops, desc = oracle_sample(w, args.cpu_heads, fwd_only=fwd_only)
+        cpu = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc + f"; {secs:.1f} s"}
+
+    in_bytes = sum(host[n].nbytes for n in names)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, "fwd" if fwd_only else "fwd+bwd",
+                                  f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB per step), no flush"),
+        "frac_of_measured_burst_peak": value / world / burst,
+        "frac_of_datasheet_peak": value / world / DATASHEET_BF16_TFLOPS,
+        "fwd_tflops": fwd_tf, "bwd_tflops": None if fwd_only else bwd_flops / ((prep_ms + main_ms + fin_ms) * 1e-3) / 1e12,
+        "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -32,7 +32,12 @@ def errors(got: np.ndarray, ref: np.ndarray):
     return max_abs, rel
 
 
-def assert_close(name, got, ref, max_abs=MAX_ABS, rel_l2=REL_L2):
+def assert_close(name, got, ref, max_abs=MAX_ABS, rel_l2=REL_L2, scale_max_abs=False):
+    """max-abs and relative-L2 bounds.  With scale_max_abs the max-abs bound is
+    multiplied by max(1, max|ref|): for stress inputs whose outputs are far from
+    unit scale, where a bf16 output ulp alone exceeds the unit-scale bound."""
+    if scale_max_abs:
+        max_abs = max_abs * max(1.0, float(np.abs(np.asarray(ref)).max()))
     ma, rl = errors(got, ref)
     assert np.isfinite(got).all(), f"{name}: non-finite values"
     assert ma <= max_abs and rl <= rel_l2, f"{name}: max_abs={ma:.3e} rel_l2={rl:.3e}"

@@ -20,7 +20,7 @@ def run_bwd(host, causal, scale=None):
     return dq, dk, dv
 
 
-def check_heads(host, dq, dk, dv, heads, H, causal, scale):
+def check_heads(host, dq, dk, dv, heads, H, causal, scale, scale_max_abs=False):
     g = {"dq": [], "dk": [], "dv": []}
     r = {"dq": [], "dk": [], "dv": []}
     for bh in heads:
@@ -31,7 +31,7 @@ def check_heads(host, dq, dk, dv, heads, H, causal, scale):
         g["dk"].append(to_f64(dk[b, h])); r["dk"].append(rk[0, 0])
         g["dv"].append(to_f64(dv[b, h])); r["dv"].append(rv[0, 0])
     for n in ("dq", "dk", "dv"):
-        assert_close(n, np.concatenate(g[n]), np.concatenate(r[n]))
+        assert_close(n, np.concatenate(g[n]), np.concatenate(r[n]), scale_max_abs=scale_max_abs)
 
 
 def test_backward_workload_sampled_heads():
@@ -57,7 +57,8 @@ def test_backward_many_heads_and_sharp_rows():
     B, H, N, d = 3, 7, 320, 128
     host, _ = make_case(B, H, N, d, 9100, k_scale=4.0, names=("q", "k", "v", "do"))
     dq, dk, dv = run_bwd(host, True)
-    check_heads(host, dq, dk, dv, range(B * H), H, True, 1.0 / np.sqrt(d))
+    # keys x4: gradients reach |x| ~ 16, where one bf16 ulp is 0.0625
+    check_heads(host, dq, dk, dv, range(B * H), H, True, 1.0 / np.sqrt(d), scale_max_abs=True)
 
 
 def test_backward_single_key_closed_form():
