@@ -23,6 +23,7 @@ FA_BF16, FA_F32 = 0, 1
 
 EXPORTS = (
     "fa_fwd", "fa_fwd_ex", "fa_fwd_workspace_size", "fa_bwd", "fa_bwd_workspace_size",
+    "fa_bwd_prepare", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc",
     "fa_get_device_status", "fa_selftest_wait_timeout", "fa_status_string", "fa_version",
 )
 
@@ -50,6 +51,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_fwd_workspace_size.argtypes = [I, I, I, I, I]
     L.fa_fwd_workspace_size.restype = Z
     L.fa_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, Z, P]
+    L.fa_bwd_prepare.argtypes = [P, P, P, I, I, I, I, P, Z, P]
+    L.fa_bwd_main.argtypes = [P, P, P, P, P, P, I, I, I, I, F, I, P, Z, P]
+    L.fa_bwd_finish.argtypes = [P, I, I, I, I, F, P, Z, P]
+    L.fa_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P]
     L.fa_bwd_workspace_size.argtypes = [I, I, I, I]
     L.fa_bwd_workspace_size.restype = Z
     L.fa_get_device_status.argtypes = [P]
@@ -57,7 +62,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_status_string.argtypes = [I]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_version.restype = ctypes.c_char_p
-    for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_get_device_status", "fa_selftest_wait_timeout"):
+    for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_prepare", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc",
+                 "fa_get_device_status", "fa_selftest_wait_timeout"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -123,6 +129,51 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, workspace, scale: fl
     _check(load_library().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
                                  _ptr(dk), _ptr(dv), B, H, N, d, scale, int(bool(causal)),
                                  _ptr(workspace), ws_bytes, _stream(stream)), "fa_bwd")
+
+
+def _ws_bytes(workspace) -> int:
+    return 0 if workspace is None else workspace.numel() * workspace.element_size()
+
+
+def fa_bwd_prepare(o, lse, dout, workspace, stream=None) -> None:
+    B, H, N, d = _bhnd(o)
+    _check(load_library().fa_bwd_prepare(_ptr(o), _ptr(lse), _ptr(dout), B, H, N, d, _ptr(workspace),
+                                         _ws_bytes(workspace), _stream(stream)), "fa_bwd_prepare")
+
+
+def fa_bwd_main(q, k, v, dout, dk, dv, causal: bool, workspace, scale: float | None = None, stream=None) -> None:
+    B, H, N, d = _bhnd(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(load_library().fa_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dk), _ptr(dv), B, H, N, d,
+                                      scale, int(bool(causal)), _ptr(workspace), _ws_bytes(workspace),
+                                      _stream(stream)), "fa_bwd_main")
+
+
+def fa_bwd_finish(dq, workspace, scale: float | None = None, stream=None) -> None:
+    B, H, N, d = _bhnd(dq)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(load_library().fa_bwd_finish(_ptr(dq), B, H, N, d, scale, _ptr(workspace), _ws_bytes(workspace),
+                                        _stream(stream)), "fa_bwd_finish")
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20   # FA_NOALLOC_SCRATCH_BYTES in include/fa.h
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float | None = None,
+                   stream=None) -> None:
+    """fa_bwd using the library's built-in scratch array instead of a workspace.
+
+    For callers that cannot allocate device memory themselves (for example a
+    plug-in whose host application owns all device allocations, or a serving
+    path that must not allocate after start-up).  Shapes needing more than
+    NOALLOC_SCRATCH_BYTES of workspace are rejected; the first call on a device
+    looks up the array's address; calls that overlap on the GPU race.
+    """
+    B, H, N, d = _bhnd(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(load_library().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                                         _ptr(dk), _ptr(dv), B, H, N, d, scale, int(bool(causal)),
+                                         _stream(stream)), "fa_bwd_noalloc")
 
 
 def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:

@@ -14,12 +14,12 @@
 
 namespace fa {
 
+constexpr int kMaxDevices = 64;
 __device__ uint32_t g_status;   // device status word (bits of DEV_*), one per device
 
 namespace {
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per bounded wait
-constexpr int kMaxDevices = 64;
 
 struct DevState {
   bool ready = false;
@@ -214,23 +214,32 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return round256(bh * N * d * 4) + 2 * round256(bh * np * 4);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-                 void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
-                 void* workspace, size_t workspace_bytes, fa_stream_t stream_) {
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+enum BwdPhase : int { PH_PREPARE = 1, PH_MAIN = 2, PH_FINISH = 4, PH_ALL = 7 };
+
+// Validates, fills the kernel arguments, and launches the requested phases.
+fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                   int causal, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   fa_status st = check_sizes(B, H, N, d, scale);
   if (st != FA_OK) return st;
   if (d != 128) return FA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+  if ((phases & PH_PREPARE) && (!aligned16(o) || !aligned16(lse) || !aligned16(dout))) return FA_ERR_ALIGN;
+  if ((phases & PH_MAIN) && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
+                             !aligned16(dk) || !aligned16(dv)))
     return FA_ERR_ALIGN;
+  if ((phases & PH_FINISH) && !aligned16(dq)) return FA_ERR_ALIGN;
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return FA_ERR_WORKSPACE;
   DevState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   using C = BwdCfg;
-  if (!ds->bwd_attr) {
+  if ((phases & PH_MAIN) && !ds->bwd_attr) {
     if (cudaFuncSetAttribute(fa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
       return FA_ERR_CUDA;
@@ -259,15 +268,85 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.wait_limit_ns = kWaitLimitNs;
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, d, N, BH, 64) || !make_map(&tk, k, d, N, BH, 128) || !make_map(&tv, v, d, N, BH, 128) ||
-      !make_map(&tdo, dout, d, N, BH, 64))
-    return FA_ERR_CUDA;
-  const int pre_blocks = ds->sms * 8;
-  fa_bwd_pre_kernel<128><<<pre_blocks, 256, 0, stream>>>(a);
-  fa_bwd_kernel<<<a.n_kb * BH, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
-  fa_bwd_dq_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
+  if (phases & PH_PREPARE) fa_bwd_pre_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
+  if (phases & PH_MAIN) {
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_map(&tq, q, d, N, BH, 64) || !make_map(&tk, k, d, N, BH, 128) ||
+        !make_map(&tv, v, d, N, BH, 128) || !make_map(&tdo, dout, d, N, BH, 64))
+      return FA_ERR_CUDA;
+    fa_bwd_kernel<<<a.n_kb * BH, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  }
+  if (phases & PH_FINISH) fa_bwd_dq_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                 void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  return bwd_impl(PH_ALL, q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+                  workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd_prepare(const void* o, const float* lse, const void* dout, int B, int H, int N, int d,
+                         void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  return bwd_impl(PH_PREPARE, nullptr, nullptr, nullptr, o, lse, dout, nullptr, nullptr, nullptr, B, H, N, d,
+                  1.0f, 0, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B,
+                      int H, int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                      fa_stream_t stream) {
+  return bwd_impl(PH_MAIN, q, k, v, nullptr, nullptr, dout, nullptr, dk, dv, B, H, N, d, scale, causal,
+                  workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd_finish(void* dq, int B, int H, int N, int d, float scale, void* workspace,
+                        size_t workspace_bytes, fa_stream_t stream) {
+  return bwd_impl(PH_FINISH, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dq, nullptr, nullptr, B, H,
+                  N, d, scale, 0, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+// ---- backward with built-in scratch (no allocation) ----
+// One fixed-size device array per device that loads the library; every
+// fa_bwd_noalloc call on that device uses it as the fa_bwd workspace.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[fa::kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (looked up once per
+// device; the host-side symbol itself is not a device address).
+fa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= fa::kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+}  // namespace
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                         int causal, fa_stream_t stream) {
+  fa_status st = check_sizes(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (need > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;   // beyond the built-in scratch
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != FA_OK) return st;
+  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, scratch,
+                FA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 fa_status fa_get_device_status(fa_stream_t stream) {

@@ -93,8 +93,54 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int B, int H, int N, int d, float scale, int causal,
                  void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
+/*
+ * The three phases fa_bwd runs, in order, on the same stream and workspace;
+ * exposed so that callers can schedule (or time) them separately.
+ *  fa_bwd_prepare: D_i = sum_c dO_ic O_ic and lse * log2(e) into the
+ *                  workspace, and zeroes the fp32 dQ accumulator there.
+ *                  Reads o, lse, dout.
+ *  fa_bwd_main:    recomputes P and dS from q, k and the prepared rows; writes
+ *                  dk, dv (bf16) and adds every dS K contribution into the dQ
+ *                  accumulator.  Reads q, k, v, dout.
+ *  fa_bwd_finish:  dq = bf16(scale * accumulator).
+ * Arguments mean what they mean for fa_bwd.  Calling them out of order, or
+ * with different sizes, gives undefined outputs (not a fault).
+ */
+fa_status fa_bwd_prepare(const void* o, const float* lse, const void* dout, int B, int H, int N, int d,
+                         void* workspace, size_t workspace_bytes, fa_stream_t stream);
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                      int B, int H, int N, int d, float scale, int causal,
+                      void* workspace, size_t workspace_bytes, fa_stream_t stream);
+fa_status fa_bwd_finish(void* dq, int B, int H, int N, int d, float scale,
+                        void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
 /* Bytes of workspace fa_bwd needs. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward without a caller-supplied workspace.  Same arguments, outputs and
+ * numerics as fa_bwd, minus the workspace pair.  The paper has no counterpart
+ * of this call; it exists for callers that cannot allocate device memory
+ * themselves -- for example a plug-in whose host application owns every
+ * device allocation through its own pool, or a serving path that must not
+ * allocate once it has started -- and so cannot hand fa_bwd a workspace.
+ *
+ * The scratch lives in one statically sized device array inside libfa.so
+ * (FA_NOALLOC_SCRATCH_BYTES bytes, held on every GPU that loads the library
+ * until the process exits).  Shapes whose fa_bwd_workspace_size() exceeds it
+ * are rejected with FA_ERR_WORKSPACE before anything is launched.  This call
+ * never allocates (no cudaMalloc, no allocating library routine).
+ *
+ * The first call on a device (with that device current) looks up the array's
+ * device address; make that first call before any stream capture.  All calls
+ * on a device share the one array and leave their contents in it: the dQ
+ * accumulator is cleared on every call, but two calls that overlap on the GPU
+ * (different streams, no ordering between them) race and give wrong results.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv,
+                         int B, int H, int N, int d, float scale, int causal, fa_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
