@@ -52,6 +52,8 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-heads", type=int, default=2, help="heads in the CPU baseline sample")
+    p.add_argument("--shape", default=None,
+                   help="B,H,N override of the workload's sizes (smaller cases for profiler captures)")
     return p.parse_args()
 
 
@@ -236,6 +238,10 @@ def workload_config(w, step: str, note: str):
 def main():
     args = parse_args()
     w = inputs.WORKLOADS[args.workload]
+    if args.shape:
+        import dataclasses
+        B_, H_, N_ = (int(x) for x in args.shape.split(","))
+        w = dataclasses.replace(w, name=f"{w.name}[{B_},{H_},{N_}]", B=B_, H=H_, N=N_)
     if args.impl == "reference":
         run_reference(args, w)
         return

@@ -20,9 +20,11 @@
 //                           dV  += P^T dO          (A = P^T bf16 from TMEM)
 //                           dK  += dS^T Q          (A = dS^T bf16 from TMEM)
 //                           dQ^T = K^T dS^T        (both operands MN-major smem)
-//                         a warpgroup with one thread per key computes P and dS;
-//                         a second warpgroup with one thread per head-dim lane
-//                         drains dQ^T into the fp32 dQ accumulator with atomic adds;
+//                         eight warps compute P and dS, two per SM sub-partition
+//                         (thread = key row, each warp 32 of the 64 query columns,
+//                         all of it elementwise); a warpgroup with one thread per
+//                         head-dim lane drains dQ^T into the fp32 dQ accumulator
+//                         with atomic adds;
 //  * fa_bwd_dq_kernel:    dQ = bf16(scale * dQacc).
 #pragma once
 
@@ -112,7 +114,8 @@ struct BwdCfg {
   static constexpr int BN = 128;               // keys per CTA
   static constexpr int BM = 64;                // queries per iteration
   static constexpr int STAGES = 3;
-  static constexpr int THREADS = 320;          // WG0 softmax, WG1 dQ drain, warp 8 MMA, warp 9 TMA
+  static constexpr int THREADS = 448;          // warps 0-7 P/dS, 8-11 dQ drain, 12 MMA, 13 TMA
+  static constexpr int PDS_THREADS = 256;
   static constexpr int KREG = 128 * 128;       // 64-col region of a 128-row tile
   static constexpr int QREG = 64 * 128;        // 64-col region of a 64-row tile
   static constexpr int KV_TILE = BN * D * 2;   // 32 KB
@@ -181,8 +184,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     mbar_init(b_s_full, 1);
     mbar_init(b_dp_full, 1);
-    mbar_init(b_p_full, 128);
-    mbar_init(b_ds_full, 128);
+    mbar_init(b_p_full, C::PDS_THREADS);
+    mbar_init(b_ds_full, C::PDS_THREADS);
     for (int b = 0; b < 2; ++b) {
       mbar_init(b_dq_full(b), 1);
       mbar_init(b_dq_free(b), 128);
@@ -191,8 +194,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     mbar_init(b_drain, 1);
     fence_mbar_init();
   }
-  if (warp == 8) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
-  if (warp == 9 && lane == 0) {
+  if (warp == 12) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  if (warp == 13 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -204,7 +207,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, args.status, args.wait_limit_ns};
 
-  if (warp == 9) {
+  if (warp == 13) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
@@ -237,7 +240,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           if ((issued >> s) & 1u) mbar_wait_quiet(b_qdo_full(s), (last_parity >> s) & 1u, 200000000ull);
       }
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(b_kv_full, 0, ctl);
@@ -317,83 +320,88 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       umma_commit(b_drain);
       mbar_wait_quiet(b_drain, 0, 200000000ull);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ P / dS warpgroup (thread = key)
-    const int rloc = warp * 32 + lane;
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ P / dS warps (thread = key, 32 query columns)
+    const int quarter = warp & 3;
+    const int chalf = warp >> 2;                   // which 32 of the 64 query columns
+    const int rloc = quarter * 32 + lane;
     const int key = k0 + rloc;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::T_S;
     const uint32_t tDP = tmem + lane_off + C::T_DP;
     const float c2 = args.scale_log2;
     const bool key_ok = key < args.N;
+    const int col0 = 32 * chalf;
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int s = it % C::STAGES;
       const uint32_t ph = it & 1;
       const int q0 = (i_begin + it) * C::BM;
       const uint8_t* st = smem + C::OFF_ST + s * C::STAGE_STRIDE;
-      const float* lse2 = reinterpret_cast<const float*>(st + C::ST_LSE);
-      const float* dvec = reinterpret_cast<const float*>(st + C::ST_DV);
+      const float* lse2 = reinterpret_cast<const float*>(st + C::ST_LSE) + col0;
+      const float* dvec = reinterpret_cast<const float*>(st + C::ST_DV) + col0;
       if (!mbar_wait_warp(b_qdo_full(s), (it / C::STAGES) & 1, ctl)) { ok = false; break; }
       if (!mbar_wait_warp(b_s_full, ph, ctl)) { ok = false; break; }
       tc_fence_after();
-      uint32_t r[64];
-      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(r));
-      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+      uint32_t r[32];
+      tmem_ld32(tS + col0, r);
       tmem_wait_ld();
-      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r));
-      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r + 32));
-      float p[64];
+      reg_fence32(r);
+      float p[32];
       // keys past the sequence end and (causal) queries before this key get P = 0
       const int cut = !key_ok ? C::BM : (args.causal ? key - q0 : 0);   // columns c < cut are masked
 #pragma unroll
-      for (int c = 0; c < 64; c += 4) {
+      for (int c = 0; c < 32; c += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);
-        p[c + 0] = ex2_approx(fmaf(__uint_as_float(r[c + 0]), c2, -l4.x));
-        p[c + 1] = ex2_approx(fmaf(__uint_as_float(r[c + 1]), c2, -l4.y));
-        p[c + 2] = ex2_approx(fmaf(__uint_as_float(r[c + 2]), c2, -l4.z));
-        p[c + 3] = ex2_approx(fmaf(__uint_as_float(r[c + 3]), c2, -l4.w));
+        const float2 x0 = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])),
+                                make_float2(c2, c2), make_float2(-l4.x, -l4.y));
+        const float2 x1 = ffma2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])),
+                                make_float2(c2, c2), make_float2(-l4.z, -l4.w));
+        p[c + 0] = ex2_approx(x0.x);
+        p[c + 1] = ex2_approx(x0.y);
+        p[c + 2] = ex2_approx(x1.x);
+        p[c + 3] = ex2_approx(x1.y);
       }
-      if (cut > 0) {
+      if (cut > col0) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < cut) p[c] = 0.f;
+        for (int c = 0; c < 32; ++c)
+          if (col0 + c < cut) p[c] = 0.f;
       }
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-      tmem_st32(tS, pk);
+      for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
+      tmem_st16(tS + (col0 >> 1), pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(b_p_full);
       // dS = P (dP - D)
       if (!mbar_wait_warp(b_dp_full, ph, ctl)) { ok = false; break; }
       tc_fence_after();
-      tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(r));
-      tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+      tmem_ld32(tDP + col0, r);
       tmem_wait_ld();
-      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r));
-      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r + 32));
+      reg_fence32(r);
 #pragma unroll
-      for (int c = 0; c < 64; c += 4) {
+      for (int c = 0; c < 32; c += 4) {
         const float4 d4 = *reinterpret_cast<const float4*>(dvec + c);
-        p[c + 0] *= __uint_as_float(r[c + 0]) - d4.x;
-        p[c + 1] *= __uint_as_float(r[c + 1]) - d4.y;
-        p[c + 2] *= __uint_as_float(r[c + 2]) - d4.z;
-        p[c + 3] *= __uint_as_float(r[c + 3]) - d4.w;
+        const float2 a = fmul2(make_float2(p[c], p[c + 1]),
+                               fsub2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), make_float2(d4.x, d4.y)));
+        const float2 b = fmul2(make_float2(p[c + 2], p[c + 3]),
+                               fsub2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), make_float2(d4.z, d4.w)));
+        p[c] = a.x; p[c + 1] = a.y; p[c + 2] = b.x; p[c + 3] = b.y;
       }
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-      tmem_st32(tDP, pk);
-      // dS^T row into the swizzled smem buffer of this iteration
+      for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
+      tmem_st16(tDP + (col0 >> 1), pk);
+      // this thread's half of the dS^T row into the swizzled smem buffer of this iteration
       const int buf = it & 1;
       if (it >= 2) {
         if (!mbar_wait_warp(b_dq_full(buf), ((it >> 1) - 1) & 1, ctl)) { ok = false; break; }
       }
       uint8_t* drow = smem + C::OFF_DS + buf * C::DS_BYTES + rloc * 128;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint4 w = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+      for (int q = 0; q < 4; ++q) {
+        const int ch = 4 * chalf + q;
+        const uint4 w = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         *reinterpret_cast<uint4*>(drow + ((ch ^ (rloc & 7)) << 4)) = w;
       }
       fence_proxy_async_smem();
@@ -401,17 +409,17 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(b_ds_full);
     }
-    // ---- epilogue: dV, dK rows -> global
+    // ---- epilogue: this thread's half of the dV, dK rows -> global
     if (ok && mbar_wait_warp(b_dkv_done, 0, ctl)) {
       tc_fence_after();
-      const size_t grow = (static_cast<size_t>(bh) * args.N + key) * D;
+      const size_t grow = (static_cast<size_t>(bh) * args.N + key) * D + 64 * chalf;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DK : C::T_DV);
+        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DK : C::T_DV) + 64 * chalf;
         __nv_bfloat16* dst = (which ? args.dk : args.dv) + grow;
         const float mul = which ? args.scale : 1.0f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
           tmem_ld32(tsrc + c * 32, v);
           tmem_wait_ld();
@@ -431,10 +439,10 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ dQ drain warpgroup (thread = head-dim lane)
-    const int dl = (warp - 4) * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    const int dl = (warp - 8) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp - 8) * 32) << 16;
     float* acc = args.dq_acc + static_cast<size_t>(bh) * args.N * D + dl;
     for (int it = 0; it < n_iter; ++it) {
       const int buf = it & 1;
@@ -460,7 +468,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);

@@ -140,9 +140,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, args.status, args.wait_limit_ns};
-
+  // Register split, taken inside each role's branch so the compiler sees which
+  // budget governs which code: 384 threads x 168 registers at launch
+  // = 128 x (224 + 224) for the softmax warpgroups + 128 x 56 for warps 8-11.
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
     if (lane == 0) {
       uint32_t kv_it = 0, tile_cnt = 0;
       bool ok = true, q_pending = false;
@@ -181,9 +184,28 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
     if (lane == 0) {
+      // descriptor of address a + off == descriptor of a, plus off / 16 (no carry:
+      // shared addresses stay below 2^18, the start field holds 14 bits of a / 16)
+      constexpr uint32_t LBO_K = 16, LBO_V = C::REGION, SBO = 1024;
       uint32_t kv_it = 0, tile_cnt = 0, p_par0 = 0, p_par1 = 0;
       bool ok = true;
+      auto issue_s = [&](uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {   // S = Q K^T
+        const uint64_t dq = sdesc_sw128(opaque_u32(q_addr), LBO_K, SBO);
+        const uint64_t dk = sdesc_sw128(opaque_u32(k_addr), LBO_K, SBO);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * C::REGION + (kk & 3) * 32) >> 4;
+          umma_ss(d_tmem, dq + off, dk + off, C::IDESC_S, kk > 0);
+        }
+      };
+      auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, bool acc) {   // O += P V
+        const uint64_t dv = sdesc_sw128(opaque_u32(v_addr), LBO_V, SBO);
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          umma_ts(d_tmem, p_tmem + kk * 8, dv + ((kk * 2048) >> 4), C::IDESC_PV, acc || (kk > 0));
+      };
       for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x, ++tile_cnt) {
         int bh, qt;
         fwd_decode_tile(args, t, bh, qt);
@@ -198,32 +220,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           ++kv_it;
           tc_fence_after();
           const uint32_t kbase = sKV + sk * C::KV_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::REGION + (kk & 3) * 32;
-            umma_ss(tmem + C::T_S0, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
-                    C::IDESC_S, kk > 0);
-          }
+          issue_s(tmem + C::T_S0, sQ, kbase);
           umma_commit(b_s_full0);
           // ---- O1 += P1 V_{j-1}
           if (j > 0) {
             if (!mbar_wait(b_p_full0 + 8, p_par1, ctl)) { ok = false; break; }
             p_par1 ^= 1;
             tc_fence_after();
-            const uint32_t vbase = sKV + sv_prev * C::KV_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < C::BN / 16; ++kk)
-              umma_ts(tmem + C::T_O1, tmem + C::T_S1 + kk * 8, sdesc_sw128(vbase + kk * 2048, C::REGION, 1024),
-                      C::IDESC_PV, (j > 1) || (kk > 0));
+            issue_pv(tmem + C::T_O1, tmem + C::T_S1, sKV + sv_prev * C::KV_BYTES, j > 1);
             umma_commit(b_kv_empty(sv_prev));
           }
           // ---- S1 = Q1 K^T
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::REGION + (kk & 3) * 32;
-            umma_ss(tmem + C::T_S1, sdesc_sw128(sQ + C::Q_HALF + off, 16, 1024),
-                    sdesc_sw128(kbase + off, 16, 1024), C::IDESC_S, kk > 0);
-          }
+          issue_s(tmem + C::T_S1, sQ + C::Q_HALF, kbase);
           umma_commit(b_s_full0 + 8);
           umma_commit(b_kv_empty(sk));
           if (j == nkv - 1) umma_commit(b_q_empty);
@@ -234,11 +242,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           if (!mbar_wait(b_p_full0, p_par0, ctl)) { ok = false; break; }
           p_par0 ^= 1;
           tc_fence_after();
-          const uint32_t vbase = sKV + sv * C::KV_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk)
-            umma_ts(tmem + C::T_O0, tmem + C::T_S0 + kk * 8, sdesc_sw128(vbase + kk * 2048, C::REGION, 1024),
-                    C::IDESC_PV, (j > 0) || (kk > 0));
+          issue_pv(tmem + C::T_O0, tmem + C::T_S0, sKV + sv * C::KV_BYTES, j > 0);
           sv_prev = sv;
         }
         if (!ok) break;
@@ -246,13 +250,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!mbar_wait(b_p_full0 + 8, p_par1, ctl)) { ok = false; break; }
         p_par1 ^= 1;
         tc_fence_after();
-        {
-          const uint32_t vbase = sKV + sv_prev * C::KV_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk)
-            umma_ts(tmem + C::T_O1, tmem + C::T_S1 + kk * 8, sdesc_sw128(vbase + kk * 2048, C::REGION, 1024),
-                    C::IDESC_PV, (nkv > 1) || (kk > 0));
-        }
+        issue_pv(tmem + C::T_O1, tmem + C::T_S1, sKV + sv_prev * C::KV_BYTES, nkv > 1);
         umma_commit(b_kv_empty(sv_prev));
         umma_commit(b_o_done);
       }
@@ -262,6 +260,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax warpgroups
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
     const int half = warp >> 2;                       // which 128-row half
     const int rloc = (warp & 3) * 32 + lane;          // TMEM lane == row within the half
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -302,15 +301,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           for (int c = 0; c < 128; ++c)
             if (c >= cut) s[c] = -INFINITY;
         }
+        // row max: four independent chains of 3-input max
         float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
+        for (int c = 4; c < 124; c += 8) {
+          mx0 = fmax3(mx0, s[c], s[c + 1]);
+          mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+          mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+          mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
         }
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        mx0 = fmax3(mx0, s[124], s[125]);
+        mx1 = fmax3(mx1, s[126], s[127]);
+        const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
         const float m_new = fmaxf(m_ref, mx);
         const bool need = (m_new - m_ref) * c2 > 8.0f;
         const bool rescale = __any_sync(0xffffffffu, need);   // warp-uniform decision
@@ -320,23 +322,33 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           l *= alpha;
           m_ref = m_new;
         }
-        const float negm = -m_ref * c2;
-        float l0 = 0.f, l1 = 0.f;
+        // p = 2^(s c2 - m c2): three of every eight pairs on the FMA pipe, the rest
+        // on the special-function unit
+        const float2 c2v = make_float2(c2, c2);
+        const float2 negm = make_float2(-m_ref * c2, -m_ref * c2);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         uint32_t pr[64];
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
-          const float p0 = ex2_approx(fmaf(s[c], c2, negm));
-          const float p1 = ex2_approx(fmaf(s[c + 1], c2, negm));
-          l0 += p0;
-          l1 += p1;
-          pr[c >> 1] = pack_bf16x2(p0, p1);
+          const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2v, negm);
+          float2 p;
+          if ((0x92u >> ((c >> 1) & 7)) & 1u) {
+            p = ex2_poly2(x);
+          } else {
+            p.x = ex2_approx(x.x);
+            p.y = ex2_approx(x.y);
+          }
+          if ((c >> 1) & 1) acc1 = fadd2(acc1, p); else acc0 = fadd2(acc0, p);
+          pr[c >> 1] = pack_bf16x2(p.x, p.y);
         }
-        l += l0 + l1;
+        const float2 acc = fadd2(acc0, acc1);
+        l += acc.x + acc.y;
         tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pr));
         tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pr + 32));
         // O rescale (after the scores are dead, to keep register pressure down).
         // Safe: S_j's commit covered every earlier MMA, including P V_{j-1} into O.
         if (rescale && j > 0) {
+          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -344,7 +356,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tmem_wait_ld();
             reg_fence32(o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            for (int e = 0; e < 32; e += 2) {
+              const float2 v = fmul2(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+              o[e] = __float_as_uint(v.x);
+              o[e + 1] = __float_as_uint(v.y);
+            }
             tmem_st32(tO + c * 32, o);
           }
         }
@@ -388,6 +404,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       if (valid) args.lse[grow] = (m_ref * c2 + __log2f(l)) * 0.69314718055994531f;
     }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");   // warps 10-11: set-up and teardown only
   }
 
   tc_fence_before();
