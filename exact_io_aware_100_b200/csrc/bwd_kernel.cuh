@@ -13,18 +13,20 @@
 // Kernels:
 //  * fa_bwd_pre_kernel:   D_i, lse_i * log2(e) (padded rows get +inf), dQacc = 0
 //  * fa_bwd_kernel:       one CTA per (batch*head, block of 128 keys), looping
-//                         over blocks of 64 queries (causal: only those that see
-//                         the keys).  Per query block five tcgen05 MMAs:
-//                           S^T  = K Q^T           (TMEM, 64 cols)
-//                           dP^T = V dO^T          (TMEM, 64 cols)
-//                           dV  += P^T dO          (A = P^T bf16 from TMEM)
-//                           dK  += dS^T Q          (A = dS^T bf16 from TMEM)
-//                           dQ^T = K^T dS^T        (both operands MN-major smem)
+//                         over blocks of 128 queries (causal: only those that see
+//                         the keys).  Per query block five 128 x 128 x 128 tcgen05
+//                         products, every operand in shared memory:
+//                           S^T  = K Q^T           (TMEM X)
+//                           dP^T = V dO^T          (TMEM X, once S^T is read out)
+//                           dV  += P^T dO          (A = P^T bf16, smem)
+//                           dK  += dS^T Q          (A = dS^T bf16, smem, same tile)
+//                           dQ^T = K^T dS^T        (TMEM Y)
 //                         eight warps compute P and dS, two per SM sub-partition
-//                         (thread = key row, each warp 32 of the 64 query columns,
-//                         all of it elementwise); a warpgroup with one thread per
-//                         head-dim lane drains dQ^T into the fp32 dQ accumulator
-//                         with atomic adds;
+//                         (thread = key row, each warp 64 of the 128 query
+//                         columns, all of it elementwise) and write them, one
+//                         after the other, into one swizzled [key][query] tile;
+//                         a warpgroup with one thread per head-dim lane drains
+//                         dQ^T into the fp32 dQ accumulator with atomic adds;
 //  * fa_bwd_dq_kernel:    dQ = bf16(scale * dQacc).
 #pragma once
 
@@ -43,9 +45,10 @@ struct BwdArgs {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   uint32_t* status;
-  int N, Np, bh;
-  int n_kb;               // ceil(N / 128)
-  int n_qb;               // ceil(N / 64)
+  int N, Np, bh;          // Np = n_qb * 128
+  int n_kb;               // ceil(N / 128) key blocks
+  int n_qb;               // ceil(N / 128) query blocks
+  int heads_per_group;    // work-item order of the main kernel
   int causal;
   float scale;
   float scale_log2;
@@ -112,32 +115,58 @@ __global__ void fa_bwd_dq_kernel(const BwdArgs a) {
 struct BwdCfg {
   static constexpr int D = 128;
   static constexpr int BN = 128;               // keys per CTA
-  static constexpr int BM = 64;                // queries per iteration
-  static constexpr int STAGES = 3;
+  static constexpr int BM = 128;               // queries per iteration
   static constexpr int THREADS = 448;          // warps 0-7 P/dS, 8-11 dQ drain, 12 MMA, 13 TMA
   static constexpr int PDS_THREADS = 256;
-  static constexpr int KREG = 128 * 128;       // 64-col region of a 128-row tile
-  static constexpr int QREG = 64 * 128;        // 64-col region of a 64-row tile
-  static constexpr int KV_TILE = BN * D * 2;   // 32 KB
-  static constexpr int Q_TILE = BM * D * 2;    // 16 KB
-  static constexpr int ST_Q = 0, ST_DO = Q_TILE, ST_LSE = 2 * Q_TILE, ST_DV = 2 * Q_TILE + BM * 4;
-  static constexpr int STAGE_BYTES = 2 * Q_TILE + 2 * BM * 4;    // 33280
-  static constexpr int STAGE_STRIDE = 33792;                     // next multiple of 1024
-  static constexpr int DS_BYTES = BN * BM * 2;                   // 16 KB
-  static constexpr int OFF_K = 0, OFF_V = KV_TILE, OFF_ST = 2 * KV_TILE;
-  static constexpr int OFF_DS = OFF_ST + STAGES * STAGE_STRIDE;
-  static constexpr int OFF_BAR = OFF_DS + 2 * DS_BYTES;
-  // barriers: kv_full, qdo_full[S], qdo_empty[S], s_full, dp_full, p_full, ds_full,
-  //           dq_full[2], dq_free[2], dkv_done, drain
-  static constexpr int N_BARS = 1 + 2 * STAGES + 4 + 4 + 2;
+  static constexpr int DRAIN_THREADS = 128;
+  // Register split (setmaxnreg).  448 threads launch with 128 registers each
+  // (four warps share a sub-partition's 16K registers); P/dS warps take 144,
+  // the MMA and TMA warps 104, the drain warps give theirs down to 72:
+  // 256 * 144 + 128 * 72 + 64 * 104 = 52736 <= 448 * 128, and per sub-partition
+  // 2 * 144 + 72 + 104 = 464 <= 512 registers per thread slot.
+  static constexpr int LAUNCH_REGS = 128;
+  static constexpr int REGS_PDS = 144, REGS_DRAIN = 72, REGS_SINGLE = 104;
+  static constexpr int REG = 128 * 128;        // one 64-column SW128 region of a 128-row bf16 tile
+  static constexpr int TILE = 2 * REG;         // a 128 x 128 bf16 tile (32 KB)
+  static constexpr int OFF_K = 0, OFF_V = TILE;
+  static constexpr int OFF_Q = 2 * TILE;       // two Q stages
+  static constexpr int OFF_DO = 4 * TILE;      // two dO stages
+  static constexpr int OFF_PS = 6 * TILE;      // P_i, then dS_i, stored [key][query]
+  static constexpr int OFF_VEC = 7 * TILE;     // per Q stage: lse2[BM] then D[BM]
+  static constexpr int VEC_BYTES = 2 * BM * 4;
+  static constexpr int OFF_BAR = OFF_VEC + 2 * VEC_BYTES;
+  static constexpr int N_BARS = 20;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int USED = OFF_MISC + 16;
+  // The opt-in maximum per block.  The kernel rounds its base up to 1 KB (SW128
+  // tiles) inside this and checks that USED still fits.
+  static constexpr int SMEM_BYTES = 232448;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t T_DV = 0, T_DK = 128, T_S = 256, T_DP = 320, T_DQ = 384;
+  static constexpr uint32_t T_DV = 0, T_DK = 128, T_X = 256, T_Y = 384;   // X: S^T, then dP^T; Y: dQ^T
   static constexpr uint32_t IDESC_SD = idesc_bf16_f32(128, BM, false, false);   // S^T, dP^T
   static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);     // dV, dK
   static constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, BM, true, true);      // dQ^T
 };
+static_assert(BwdCfg::USED + 768 <= BwdCfg::SMEM_BYTES, "shared memory plan");
+static_assert(BwdCfg::PDS_THREADS * BwdCfg::REGS_PDS + BwdCfg::DRAIN_THREADS * BwdCfg::REGS_DRAIN +
+                  64 * BwdCfg::REGS_SINGLE <= BwdCfg::THREADS * BwdCfg::LAUNCH_REGS,
+              "register split exceeds the registers the block launches with");
+static_assert(2 * BwdCfg::REGS_PDS + BwdCfg::REGS_DRAIN + BwdCfg::REGS_SINGLE <= 512,
+              "register split exceeds a sub-partition");
+
+// Work item x -> (head, key block).  Heads are taken in groups of
+// heads_per_group; inside a group the key blocks with the most query blocks
+// come first (causal), so the dQ accumulators being added to at any time are
+// those of a few heads and stay in L2.
+__device__ __forceinline__ void bwd_decode(const BwdArgs& a, int x, int& bh, int& kb) {
+  const int per_group = a.heads_per_group * a.n_kb;
+  const int g = x / per_group;
+  const int r = x - g * per_group;
+  const int h0 = g * a.heads_per_group;
+  const int gh = min(a.heads_per_group, a.bh - h0);
+  kb = r / gh;
+  bh = h0 + (r - kb * gh);
+}
 
 __global__ void __launch_bounds__(BwdCfg::THREADS, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -145,51 +174,66 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               const BwdArgs args) {
   using C = BwdCfg;
   constexpr int D = C::D;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sbase = smem_u32(smem);
-  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
-  auto sStage = [&](int s) { return sbase + C::OFF_ST + s * C::STAGE_STRIDE; };
-  auto sDS = [&](int b) { return sbase + C::OFF_DS + b * C::DS_BYTES; };
+  extern __shared__ __align__(16) uint8_t smem_raw[];   // only 16 B promised: the 1 KB rounding below is real
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  if (pad + C::USED > static_cast<uint32_t>(C::SMEM_BYTES)) {   // buffers do not fit: report, touch nothing
+    if (threadIdx.x == 0) atomicOr(args.status, DEV_SMEM);
+    return;
+  }
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw + pad;
+  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sPS = sbase + C::OFF_PS;
+  auto sQ = [&](int s) { return sbase + C::OFF_Q + s * C::TILE; };
+  auto sDO = [&](int s) { return sbase + C::OFF_DO + s * C::TILE; };
+  auto sVec = [&](int s) { return sbase + C::OFF_VEC + s * C::VEC_BYTES; };
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  const uint32_t b_kv_full = bar0;
-  auto b_qdo_full = [&](int s) { return bar0 + 8 + 8 * s; };
-  auto b_qdo_empty = [&](int s) { return bar0 + 8 + 8 * C::STAGES + 8 * s; };
-  const uint32_t b_s_full = bar0 + 8 + 16 * C::STAGES;
-  const uint32_t b_dp_full = b_s_full + 8;
-  const uint32_t b_p_full = b_s_full + 16;
-  const uint32_t b_ds_full = b_s_full + 24;
-  auto b_dq_full = [&](int b) { return b_s_full + 32 + 8 * b; };
-  auto b_dq_free = [&](int b) { return b_s_full + 48 + 8 * b; };
-  const uint32_t b_dkv_done = b_s_full + 64;
-  const uint32_t b_drain = b_s_full + 72;
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  const uint32_t b_kv_full = bar(0);
+  auto b_q_full = [&](int s) { return bar(1 + s); };
+  auto b_q_empty = [&](int s) { return bar(3 + s); };
+  auto b_do_full = [&](int s) { return bar(5 + s); };
+  auto b_do_empty = [&](int s) { return bar(7 + s); };
+  const uint32_t b_s_full = bar(9);      // S_i in X
+  const uint32_t b_dp_full = bar(10);    // dP_i in X
+  const uint32_t b_x_free = bar(11);     // X read out (twice per query block: S, then dP)
+  const uint32_t b_p_ready = bar(12);    // P_i in the P/dS tile
+  const uint32_t b_dv_done = bar(13);    // dV_i done reading P_i
+  const uint32_t b_ds_ready = bar(14);   // dS_i in the P/dS tile
+  const uint32_t b_ps_free = bar(15);    // dK_i, dQ_i done reading dS_i
+  const uint32_t b_dq_full = bar(16);    // dQ^T_i in Y
+  const uint32_t b_dq_free = bar(17);    // Y read out
+  const uint32_t b_dkv_done = bar(18);
+  const uint32_t b_drain = bar(19);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // work item: key blocks with the most query blocks first (causal), then heads
-  const int kb = static_cast<int>(blockIdx.x) / args.bh;
-  const int bh = static_cast<int>(blockIdx.x) % args.bh;
+  int bh, kb;
+  bwd_decode(args, static_cast<int>(blockIdx.x), bh, kb);
   const int k0 = kb * C::BN;
-  const int i_begin = args.causal ? (k0 / C::BM) : 0;
+  const int i_begin = args.causal ? kb : 0;          // query blocks that see these keys (BM == BN)
   const int n_iter = args.n_qb - i_begin;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0u;
     mbar_init(b_kv_full, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(b_qdo_full(s), 1);
-      mbar_init(b_qdo_empty(s), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(b_q_full(s), 1);
+      mbar_init(b_q_empty(s), 1);
+      mbar_init(b_do_full(s), 1);
+      mbar_init(b_do_empty(s), 1);
     }
     mbar_init(b_s_full, 1);
     mbar_init(b_dp_full, 1);
-    mbar_init(b_p_full, C::PDS_THREADS);
-    mbar_init(b_ds_full, C::PDS_THREADS);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(b_dq_full(b), 1);
-      mbar_init(b_dq_free(b), 128);
-    }
+    mbar_init(b_x_free, C::PDS_THREADS);
+    mbar_init(b_p_ready, C::PDS_THREADS);
+    mbar_init(b_dv_done, 1);
+    mbar_init(b_ds_ready, C::PDS_THREADS);
+    mbar_init(b_ps_free, 1);
+    mbar_init(b_dq_full, 1);
+    mbar_init(b_dq_free, C::DRAIN_THREADS);
     mbar_init(b_dkv_done, 1);
     mbar_init(b_drain, 1);
     fence_mbar_init();
@@ -209,213 +253,227 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   if (warp == 13) {
     // ------------------------------------------------------------ TMA producer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;");
     if (lane == 0) {
       bool ok = true;
-      uint32_t issued = 0, last_parity = 0;      // per-stage bit masks
-      mbar_expect_tx(b_kv_full, 2 * C::KV_TILE);
+      int q_last[2] = {-1, -1}, do_last[2] = {-1, -1};     // last query block loaded into each stage
+      mbar_expect_tx(b_kv_full, 2 * C::TILE);
       for (int r = 0; r < 2; ++r) {
-        tma_load_3d(sK + r * C::KREG, &tm_k, b_kv_full, r * 64, k0, bh);
-        tma_load_3d(sV + r * C::KREG, &tm_v, b_kv_full, r * 64, k0, bh);
+        tma_load_3d(sK + r * C::REG, &tm_k, b_kv_full, r * 64, k0, bh);
+        tma_load_3d(sV + r * C::REG, &tm_v, b_kv_full, r * 64, k0, bh);
       }
       for (int it = 0; it < n_iter; ++it) {
-        const int s = it % C::STAGES;
-        const uint32_t round = it / C::STAGES;
-        if (round > 0 && !mbar_wait(b_qdo_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
+        const int s = it & 1;
+        const uint32_t round = static_cast<uint32_t>(it) >> 1;
         const int q0 = (i_begin + it) * C::BM;
-        const uint32_t st = sStage(s);
-        mbar_expect_tx(b_qdo_full(s), C::STAGE_BYTES);
-        for (int r = 0; r < 2; ++r) {
-          tma_load_3d(st + C::ST_Q + r * C::QREG, &tm_q, b_qdo_full(s), r * 64, q0, bh);
-          tma_load_3d(st + C::ST_DO + r * C::QREG, &tm_do, b_qdo_full(s), r * 64, q0, bh);
-        }
+        // Q_i with its lse2 and D rows; the stage is released after dK_i
+        if (round > 0 && !mbar_wait(b_q_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
+        mbar_expect_tx(b_q_full(s), C::TILE + C::VEC_BYTES);
+        for (int r = 0; r < 2; ++r) tma_load_3d(sQ(s) + r * C::REG, &tm_q, b_q_full(s), r * 64, q0, bh);
         const size_t voff = static_cast<size_t>(bh) * args.Np + q0;
-        bulk_load(st + C::ST_LSE, args.lse2 + voff, C::BM * 4, b_qdo_full(s));
-        bulk_load(st + C::ST_DV, args.dvec + voff, C::BM * 4, b_qdo_full(s));
-        issued |= 1u << s;
-        last_parity = (last_parity & ~(1u << s)) | ((round & 1u) << s);
+        bulk_load(sVec(s), args.lse2 + voff, C::BM * 4, b_q_full(s));
+        bulk_load(sVec(s) + C::BM * 4, args.dvec + voff, C::BM * 4, b_q_full(s));
+        q_last[s] = it;
+        // dO_i; the stage is released after dV_i
+        if (round > 0 && !mbar_wait(b_do_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
+        mbar_expect_tx(b_do_full(s), C::TILE);
+        for (int r = 0; r < 2; ++r) tma_load_3d(sDO(s) + r * C::REG, &tm_do, b_do_full(s), r * 64, q0, bh);
+        do_last[s] = it;
       }
-      if (!ok) {
+      if (!ok) {       // let the loads in flight land before the CTA exits
         mbar_wait_quiet(b_kv_full, 0, 200000000ull);
-        for (int s = 0; s < C::STAGES; ++s)
-          if ((issued >> s) & 1u) mbar_wait_quiet(b_qdo_full(s), (last_parity >> s) & 1u, 200000000ull);
+        for (int s = 0; s < 2; ++s) {
+          if (q_last[s] >= 0) mbar_wait_quiet(b_q_full(s), (q_last[s] >> 1) & 1, 200000000ull);
+          if (do_last[s] >= 0) mbar_wait_quiet(b_do_full(s), (do_last[s] >> 1) & 1, 200000000ull);
+        }
       }
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;");
     if (lane == 0) {
+      // Descriptors are built once; a K step adds to the start-address field:
+      // K-major tiles advance 32 B inside a 128-B row and switch region every
+      // four steps, MN-major tiles advance 16 rows (2 KB).
+      const uint64_t dK_k = sdesc_sw128(sK, 16, 1024), dV_k = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dK_mn = sdesc_sw128(sK, C::REG, 1024);
+      const uint64_t dPS_k = sdesc_sw128(sPS, 16, 1024), dPS_mn = sdesc_sw128(sPS, C::REG, 1024);
+      const uint64_t dQ_k0 = sdesc_sw128(sQ(0), 16, 1024), dQ_k1 = sdesc_sw128(sQ(1), 16, 1024);
+      const uint64_t dQ_mn0 = sdesc_sw128(sQ(0), C::REG, 1024), dQ_mn1 = sdesc_sw128(sQ(1), C::REG, 1024);
+      const uint64_t dO_k0 = sdesc_sw128(sDO(0), 16, 1024), dO_k1 = sdesc_sw128(sDO(1), 16, 1024);
+      const uint64_t dO_mn0 = sdesc_sw128(sDO(0), C::REG, 1024), dO_mn1 = sdesc_sw128(sDO(1), C::REG, 1024);
+      auto kstep = [](int kk) { return static_cast<uint64_t>((kk >> 2) * (C::REG >> 4) + (kk & 3) * 2); };
+      auto mnstep = [](int kk) { return static_cast<uint64_t>(kk * (2048 >> 4)); };
+      // S^T = K Q^T and dP^T = V dO^T (both operands K-major), into X
+      auto issue_kmaj = [&](uint64_t a, uint64_t b) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) umma_ss(tmem + C::T_X, a + kstep(kk), b + kstep(kk), C::IDESC_SD, kk > 0);
+      };
+      // dV += P^T dO, dK += dS^T Q: A = the P/dS tile (K-major), B MN-major
+      auto issue_kv = [&](uint32_t d_tmem, uint64_t b, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < C::BM / 16; ++kk)
+          umma_ss(d_tmem, dPS_k + kstep(kk), b + mnstep(kk), C::IDESC_KV, (acc || kk > 0) ? 1u : 0u);
+      };
       bool ok = mbar_wait(b_kv_full, 0, ctl);
-      tc_fence_after();
-      auto issue_s = [&](int s) {       // S^T = K Q^T
-        const uint32_t qb = sStage(s) + C::ST_Q;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * C::KREG + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * C::QREG + (kk & 3) * 32;
-          umma_ss(tmem + C::T_S, sdesc_sw128(sK + ko, 16, 1024), sdesc_sw128(qb + qo, 16, 1024),
-                  C::IDESC_SD, kk > 0);
-        }
-        umma_commit(b_s_full);
-      };
-      auto issue_dp = [&](int s) {      // dP^T = V dO^T
-        const uint32_t db = sStage(s) + C::ST_DO;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * C::KREG + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * C::QREG + (kk & 3) * 32;
-          umma_ss(tmem + C::T_DP, sdesc_sw128(sV + ko, 16, 1024), sdesc_sw128(db + qo, 16, 1024),
-                  C::IDESC_SD, kk > 0);
-        }
-        umma_commit(b_dp_full);
-      };
+      // prologue: S_0, and dP_0 once S_0 has been read out of X
+      if (ok) ok = mbar_wait(b_q_full(0), 0, ctl);
       if (ok) {
-        if (!mbar_wait(b_qdo_full(0), 0, ctl)) ok = false;
         tc_fence_after();
+        issue_kmaj(dK_k, dQ_k0);
+        umma_commit(b_s_full);
+        ok = mbar_wait(b_x_free, 0, ctl) && mbar_wait(b_do_full(0), 0, ctl);
       }
       if (ok) {
-        issue_s(0);
-        issue_dp(0);
+        tc_fence_after();
+        issue_kmaj(dV_k, dO_k0);
+        umma_commit(b_dp_full);
       }
       for (int it = 0; it < n_iter && ok; ++it) {
-        const int s = it % C::STAGES;
-        const uint32_t ph = it & 1;
-        // dV += P^T dO
-        if (!mbar_wait(b_p_full, ph, ctl)) { ok = false; break; }
+        const int s = it & 1;
+        const uint32_t ph = static_cast<uint32_t>(it) & 1;
+        const bool more = it + 1 < n_iter;
+        const uint32_t ph1 = (static_cast<uint32_t>(it + 1) >> 1) & 1;   // round parity of block it + 1
+        // dV += P_i^T dO_i
+        if (!mbar_wait(b_p_ready, ph, ctl)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t db = sStage(s) + C::ST_DO;
-        const uint32_t qb = sStage(s) + C::ST_Q;
-#pragma unroll
-        for (int kk = 0; kk < C::BM / 16; ++kk)
-          umma_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, sdesc_sw128(db + kk * 2048, C::QREG, 1024),
-                  C::IDESC_KV, (it > 0) || (kk > 0));
-        // next S^T
-        const int s1 = (it + 1) % C::STAGES;
-        if (it + 1 < n_iter) {
-          if (!mbar_wait(b_qdo_full(s1), ((it + 1) / C::STAGES) & 1, ctl)) { ok = false; break; }
+        issue_kv(tmem + C::T_DV, s ? dO_mn1 : dO_mn0, it > 0);
+        umma_commit(b_dv_done);
+        umma_commit(b_do_empty(s));
+        // S_{i+1}, once dP_i has been read out of X
+        if (more) {
+          if (!mbar_wait(b_x_free, 1, ctl) || !mbar_wait(b_q_full(s ^ 1), ph1, ctl)) { ok = false; break; }
           tc_fence_after();
-          issue_s(s1);
+          issue_kmaj(dK_k, s ? dQ_k0 : dQ_k1);
+          umma_commit(b_s_full);
         }
-        // dK += dS^T Q
-        if (!mbar_wait(b_ds_full, ph, ctl)) { ok = false; break; }
+        // dK += dS_i^T Q_i, dQ^T_i = K^T dS_i^T
+        if (!mbar_wait(b_ds_ready, ph, ctl)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::BM / 16; ++kk)
-          umma_ts(tmem + C::T_DK, tmem + C::T_DP + kk * 8, sdesc_sw128(qb + kk * 2048, C::QREG, 1024),
-                  C::IDESC_KV, (it > 0) || (kk > 0));
-        umma_commit(b_qdo_empty(s));
-        // dQ^T = K^T dS^T
-        const int buf = it & 1;
-        if (it >= 2) {
-          if (!mbar_wait(b_dq_free(buf), ((it >> 1) - 1) & 1, ctl)) { ok = false; break; }
+        issue_kv(tmem + C::T_DK, s ? dQ_mn1 : dQ_mn0, it > 0);
+        umma_commit(b_q_empty(s));
+        if (it > 0) {
+          if (!mbar_wait(b_dq_free, ph ^ 1u, ctl)) { ok = false; break; }
           tc_fence_after();
         }
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          umma_ss(tmem + C::T_DQ + buf * C::BM, sdesc_sw128(sK + kk * 2048, C::KREG, 1024),
-                  sdesc_sw128(sDS(buf) + kk * 2048, C::QREG, 1024), C::IDESC_Q, kk > 0);
-        umma_commit(b_dq_full(buf));
-        // next dP^T
-        if (it + 1 < n_iter) issue_dp(s1);
+          umma_ss(tmem + C::T_Y, dK_mn + mnstep(kk), dPS_mn + mnstep(kk), C::IDESC_Q, kk > 0);
+        umma_commit(b_dq_full);
+        umma_commit(b_ps_free);
+        // dP_{i+1}, once S_{i+1} has been read out of X
+        if (more) {
+          if (!mbar_wait(b_x_free, 0, ctl) || !mbar_wait(b_do_full(s ^ 1), ph1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          issue_kmaj(dV_k, s ? dO_k0 : dO_k1);
+          umma_commit(b_dp_full);
+        }
       }
       if (ok) umma_commit(b_dkv_done);
       umma_commit(b_drain);
       mbar_wait_quiet(b_drain, 0, 200000000ull);
     }
   } else if (warp < 8) {
-    // ------------------------------------------------------------ P / dS warps (thread = key, 32 query columns)
+    // ------------------------------------------------------------ P / dS warps (thread = key, 64 query columns)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 144;");
     const int quarter = warp & 3;
-    const int chalf = warp >> 2;                   // which 32 of the 64 query columns
-    const int rloc = quarter * 32 + lane;
+    const int ch = warp >> 2;                       // which 64 of the 128 query columns
+    const int rloc = quarter * 32 + lane;           // key row in the block == TMEM lane
     const int key = k0 + rloc;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::T_S;
-    const uint32_t tDP = tmem + lane_off + C::T_DP;
+    const uint32_t tX = tmem + lane_off + C::T_X + 64 * ch;
     const float c2 = args.scale_log2;
     const bool key_ok = key < args.N;
-    const int col0 = 32 * chalf;
+    // this thread's half row of the P / dS tile: region ch, row rloc; 16-byte
+    // chunk j of the row sits at chunk j ^ (row & 7) (128-byte swizzle)
+    uint8_t* prow = smem + C::OFF_PS + ch * C::REG + rloc * 128;
+    const int sw = rloc & 7;
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
-      const int s = it % C::STAGES;
-      const uint32_t ph = it & 1;
+      const int s = it & 1;
+      const uint32_t ph = static_cast<uint32_t>(it) & 1;
       const int q0 = (i_begin + it) * C::BM;
-      const uint8_t* st = smem + C::OFF_ST + s * C::STAGE_STRIDE;
-      const float* lse2 = reinterpret_cast<const float*>(st + C::ST_LSE) + col0;
-      const float* dvec = reinterpret_cast<const float*>(st + C::ST_DV) + col0;
-      if (!mbar_wait_warp(b_qdo_full(s), (it / C::STAGES) & 1, ctl)) { ok = false; break; }
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * C::VEC_BYTES) + 64 * ch;
+      const float* dvec = lse2 + C::BM;
+      if (!mbar_wait_warp(b_q_full(s), (static_cast<uint32_t>(it) >> 1) & 1, ctl)) { ok = false; break; }
       if (!mbar_wait_warp(b_s_full, ph, ctl)) { ok = false; break; }
       tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(tS + col0, r);
-      tmem_wait_ld();
-      reg_fence32(r);
-      float p[32];
-      // keys past the sequence end and (causal) queries before this key get P = 0
+      float p[64];
+      {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(tX, ra);
+        tmem_ld32(tX + 32, rb);
+        tmem_wait_ld();
+        reg_fence32(ra);
+        reg_fence32(rb);
+        tc_fence_before();
+        mbar_arrive(b_x_free);
+        const float2 c2v = make_float2(c2, c2);
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float2 la = *reinterpret_cast<const float2*>(lse2 + c);
+          const float2 lb = *reinterpret_cast<const float2*>(lse2 + 32 + c);
+          const float2 xa = ffma2(make_float2(__uint_as_float(ra[c]), __uint_as_float(ra[c + 1])), c2v,
+                                  make_float2(-la.x, -la.y));
+          const float2 xb = ffma2(make_float2(__uint_as_float(rb[c]), __uint_as_float(rb[c + 1])), c2v,
+                                  make_float2(-lb.x, -lb.y));
+          p[c] = ex2_approx(xa.x);
+          p[c + 1] = ex2_approx(xa.y);
+          p[32 + c] = ex2_approx(xb.x);
+          p[32 + c + 1] = ex2_approx(xb.y);
+        }
+      }
+      // keys past the sequence end, and (causal) queries before this key, get P = 0
       const int cut = !key_ok ? C::BM : (args.causal ? key - q0 : 0);   // columns c < cut are masked
+      if (cut > 64 * ch) {
 #pragma unroll
-      for (int c = 0; c < 32; c += 4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);
-        const float2 x0 = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])),
-                                make_float2(c2, c2), make_float2(-l4.x, -l4.y));
-        const float2 x1 = ffma2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])),
-                                make_float2(c2, c2), make_float2(-l4.z, -l4.w));
-        p[c + 0] = ex2_approx(x0.x);
-        p[c + 1] = ex2_approx(x0.y);
-        p[c + 2] = ex2_approx(x1.x);
-        p[c + 3] = ex2_approx(x1.y);
+        for (int c = 0; c < 64; ++c)
+          if (64 * ch + c < cut) p[c] = 0.f;
       }
-      if (cut > col0) {
+      uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (col0 + c < cut) p[c] = 0.f;
-      }
-      uint32_t pk[16];
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
+      if (it > 0 && !mbar_wait_warp(b_ps_free, ph ^ 1u, ctl)) { ok = false; break; }
 #pragma unroll
-      for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-      tmem_st16(tS + (col0 >> 1), pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(b_p_full);
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4*>(prow + ((j ^ sw) << 4)) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      fence_proxy_async_smem();
+      mbar_arrive(b_p_ready);
       // dS = P (dP - D)
       if (!mbar_wait_warp(b_dp_full, ph, ctl)) { ok = false; break; }
       tc_fence_after();
-      tmem_ld32(tDP + col0, r);
-      tmem_wait_ld();
-      reg_fence32(r);
 #pragma unroll
-      for (int c = 0; c < 32; c += 4) {
-        const float4 d4 = *reinterpret_cast<const float4*>(dvec + c);
-        const float2 a = fmul2(make_float2(p[c], p[c + 1]),
-                               fsub2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), make_float2(d4.x, d4.y)));
-        const float2 b = fmul2(make_float2(p[c + 2], p[c + 3]),
-                               fsub2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), make_float2(d4.z, d4.w)));
-        p[c] = a.x; p[c + 1] = a.y; p[c + 2] = b.x; p[c + 3] = b.y;
-      }
+      for (int h = 0; h < 2; ++h) {      // two 32-column halves (register budget)
+        uint32_t ra[32];
+        tmem_ld32(tX + 32 * h, ra);
+        tmem_wait_ld();
+        reg_fence32(ra);
+        if (h == 1) {
+          tc_fence_before();
+          mbar_arrive(b_x_free);
+        }
 #pragma unroll
-      for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-      tmem_st16(tDP + (col0 >> 1), pk);
-      // this thread's half of the dS^T row into the swizzled smem buffer of this iteration
-      const int buf = it & 1;
-      if (it >= 2) {
-        if (!mbar_wait_warp(b_dq_full(buf), ((it >> 1) - 1) & 1, ctl)) { ok = false; break; }
+        for (int c = 0; c < 32; c += 2) {
+          const float2 dd = *reinterpret_cast<const float2*>(dvec + 32 * h + c);
+          const float2 g = fmul2(make_float2(p[32 * h + c], p[32 * h + c + 1]),
+                                 fsub2(make_float2(__uint_as_float(ra[c]), __uint_as_float(ra[c + 1])), dd));
+          pk[16 * h + (c >> 1)] = pack_bf16x2(g.x, g.y);
+        }
       }
-      uint8_t* drow = smem + C::OFF_DS + buf * C::DS_BYTES + rloc * 128;
+      if (!mbar_wait_warp(b_dv_done, ph, ctl)) { ok = false; break; }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int ch = 4 * chalf + q;
-        const uint4 w = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        *reinterpret_cast<uint4*>(drow + ((ch ^ (rloc & 7)) << 4)) = w;
-      }
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4*>(prow + ((j ^ sw) << 4)) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
       fence_proxy_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(b_ds_full);
+      mbar_arrive(b_ds_ready);
     }
     // ---- epilogue: this thread's half of the dV, dK rows -> global
     if (ok && mbar_wait_warp(b_dkv_done, 0, ctl)) {
       tc_fence_after();
-      const size_t grow = (static_cast<size_t>(bh) * args.N + key) * D + 64 * chalf;
+      const size_t grow = (static_cast<size_t>(bh) * args.N + key) * D + 64 * ch;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DK : C::T_DV) + 64 * chalf;
+        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DK : C::T_DV) + 64 * ch;
         __nv_bfloat16* dst = (which ? args.dk : args.dv) + grow;
         const float mul = which ? args.scale : 1.0f;
 #pragma unroll
@@ -439,30 +497,40 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
     }
-  } else if (warp < 12) {
-    // ------------------------------------------------------------ dQ drain warpgroup (thread = head-dim lane)
+  } else {
+    // ------------------------------------------------------------ dQ drain (thread = head-dim lane)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
     const int dl = (warp - 8) * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>((warp - 8) * 32) << 16;
+    const uint32_t tY = tmem + (static_cast<uint32_t>((warp - 8) * 32) << 16) + C::T_Y;
     float* acc = args.dq_acc + static_cast<size_t>(bh) * args.N * D + dl;
     for (int it = 0; it < n_iter; ++it) {
-      const int buf = it & 1;
-      if (!mbar_wait_warp(b_dq_full(buf), (it >> 1) & 1, ctl)) break;
+      if (!mbar_wait_warp(b_dq_full, static_cast<uint32_t>(it) & 1, ctl)) break;
       tc_fence_after();
-      uint32_t r[64];
-      const uint32_t tq = tmem + lane_off + C::T_DQ + buf * C::BM;
-      tmem_ld32(tq, *reinterpret_cast<uint32_t(*)[32]>(r));
-      tmem_ld32(tq + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-      tmem_wait_ld();
-      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r));
-      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r + 32));
-      tc_fence_before();
-      mbar_arrive(b_dq_free(buf));
       const int q0 = (i_begin + it) * C::BM;
       const int nq = min(C::BM, args.N - q0);
-      float* a_row = acc + static_cast<size_t>(q0) * D;
 #pragma unroll
-      for (int c = 0; c < 64; ++c)
-        if (c < nq) red_add_f32(a_row + static_cast<size_t>(c) * D, __uint_as_float(r[c]));
+      for (int h = 0; h < 2; ++h) {      // two 64-column halves (register budget); Y is free after the second load
+        uint32_t r[64];
+        tmem_ld32(tY + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(r));
+        tmem_ld32(tY + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        tmem_wait_ld();
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r));
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        if (h == 1) {
+          tc_fence_before();
+          mbar_arrive(b_dq_free);
+        }
+        float* a_row = acc + static_cast<size_t>(q0 + 64 * h) * D;
+        const int nh = nq - 64 * h;      // valid rows in this half (may be <= 0)
+        if (nh >= 64) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) red_add_f32(a_row + static_cast<size_t>(c) * D, __uint_as_float(r[c]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < nh) red_add_f32(a_row + static_cast<size_t>(c) * D, __uint_as_float(r[c]));
+        }
+      }
     }
   }
 

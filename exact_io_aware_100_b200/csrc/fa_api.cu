@@ -115,12 +115,22 @@ __global__ void wait_probe_kernel(uint32_t* status, unsigned long long limit_ns)
   __syncthreads();
 }
 
+// The register splits inside the kernels (setmaxnreg) are computed for the
+// register count each kernel is launched with; a build that compiled to a
+// different count would make a setmaxnreg.inc wait forever, so such a kernel
+// is never launched.
+bool launch_regs_are(const void* fn, int regs) {
+  cudaFuncAttributes fa_attr;
+  return cudaFuncGetAttributes(&fa_attr, fn) == cudaSuccess && fa_attr.numRegs == regs;
+}
+
 template <int D>
 fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, void* o, float* lse,
                      int BH, int N, float scale, int causal, int o_f32, cudaStream_t stream) {
   using C = FwdCfg<D>;
   bool& attr = (D == 64) ? ds->fwd_attr64 : ds->fwd_attr128;
   if (!attr) {
+    if (!launch_regs_are(reinterpret_cast<const void*>(fa_fwd_kernel<D>), C::LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(fa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
       return FA_ERR_CUDA;
@@ -210,7 +220,7 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
   const size_t bh = static_cast<size_t>(B) * H;
-  const size_t np = (static_cast<size_t>(N) + 63) / 64 * 64;
+  const size_t np = (static_cast<size_t>(N) + 127) / 128 * 128;
   return round256(bh * N * d * 4) + 2 * round256(bh * np * 4);
 }
 
@@ -240,6 +250,7 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   if ((st = device_state(&ds)) != FA_OK) return st;
   using C = BwdCfg;
   if ((phases & PH_MAIN) && !ds->bwd_attr) {
+    if (!launch_regs_are(reinterpret_cast<const void*>(fa_bwd_kernel), C::LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(fa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess)
       return FA_ERR_CUDA;
@@ -247,7 +258,7 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   }
   const int BH = B * H;
   BwdArgs a;
-  const size_t np = (static_cast<size_t>(N) + 63) / 64 * 64;
+  const size_t np = (static_cast<size_t>(N) + 127) / 128 * 128;
   uint8_t* w = static_cast<uint8_t*>(workspace);
   a.dq_acc = reinterpret_cast<float*>(w);
   a.lse2 = reinterpret_cast<float*>(w + round256(static_cast<size_t>(BH) * N * d * 4));
@@ -263,7 +274,10 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   a.Np = static_cast<int>(np);
   a.bh = BH;
   a.n_kb = (N + 127) / 128;
-  a.n_qb = (N + 63) / 64;
+  a.n_qb = (N + 127) / 128;
+  // enough heads per group to fill the GPU about twice over with key blocks
+  const int want = (2 * ds->sms + a.n_kb - 1) / a.n_kb;
+  a.heads_per_group = want < 1 ? 1 : (want > BH ? BH : want);
   a.causal = causal ? 1 : 0;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
@@ -271,8 +285,8 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   if (phases & PH_PREPARE) fa_bwd_pre_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
   if (phases & PH_MAIN) {
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_map(&tq, q, d, N, BH, 64) || !make_map(&tk, k, d, N, BH, 128) ||
-        !make_map(&tv, v, d, N, BH, 128) || !make_map(&tdo, dout, d, N, BH, 64))
+    if (!make_map(&tq, q, d, N, BH, 128) || !make_map(&tk, k, d, N, BH, 128) ||
+        !make_map(&tv, v, d, N, BH, 128) || !make_map(&tdo, dout, d, N, BH, 128))
       return FA_ERR_CUDA;
     fa_bwd_kernel<<<a.n_kb * BH, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
   }
@@ -354,7 +368,8 @@ fa_status fa_get_device_status(fa_stream_t stream) {
   uint32_t v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
   if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-  return (v & DEV_TIMEOUT) ? FA_ERR_TIMEOUT : FA_OK;
+  if (v & DEV_TIMEOUT) return FA_ERR_TIMEOUT;
+  return (v & DEV_SMEM) ? FA_ERR_CUDA : FA_OK;
 }
 
 fa_status fa_selftest_wait_timeout(uint64_t timeout_ns, fa_stream_t stream) {

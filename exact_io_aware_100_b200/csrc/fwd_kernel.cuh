@@ -59,6 +59,10 @@ struct FwdCfg {
   static constexpr int KV_BYTES = BN * D * 2;     // bytes of one K or V block
   static constexpr int STAGES = (D == 128) ? 4 : 8;
   static constexpr int THREADS = 384;
+  // Register split (setmaxnreg): 384 threads launch with 168 registers each
+  // (three warps per sub-partition); the eight softmax warps take 224, the
+  // other four give theirs down to 56: 256 * 224 + 128 * 56 = 384 * 168.
+  static constexpr int LAUNCH_REGS = 168;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
   // shared-memory layout (offsets from a 1024-aligned base)

@@ -19,6 +19,7 @@ namespace fa {
 enum : uint32_t {
   DEV_OK = 0u,
   DEV_TIMEOUT = 1u,      // a bounded mbarrier wait gave up
+  DEV_SMEM = 2u,         // a kernel's shared-memory plan did not fit its allocation
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -145,7 +145,9 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device.  Returns FA_ERR_TIMEOUT if any kernel since the last call
- * gave up a bounded wait, FA_ERR_CUDA if the synchronisation failed, else FA_OK.
+ * gave up a bounded wait, FA_ERR_CUDA if the synchronisation failed or a
+ * kernel found its shared-memory allocation too small for its buffers (it then
+ * did no work), else FA_OK.
  */
 fa_status fa_get_device_status(fa_stream_t stream);
 

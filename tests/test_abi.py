@@ -76,7 +76,7 @@ def test_argument_validation_without_device(lib):
 def test_workspace_sizes(lib):
     assert lib.fa_fwd_workspace_size(1, 1, 128, 64, 0) == 0
     assert lib.fa_fwd_workspace_size(1, 1, 128, 64, 1) == 3 * 128 * 64 * 2
-    # dQ accumulator (fp32) + lse and D for rows padded to a multiple of 64
+    # dQ accumulator (fp32) + lse and D for rows padded to a multiple of 128
     assert lib.fa_bwd_workspace_size(4, 16, 4096, 128) == 4 * 16 * 4096 * 128 * 4 + 2 * 4 * 16 * 4096 * 4
     assert lib.fa_bwd_workspace_size(1, 1, 100, 128) == 100 * 128 * 4 + 2 * 512
 
