@@ -15,16 +15,17 @@
 //  * fa_bwd_kernel:       one CTA per (batch*head, block of 128 keys), looping
 //                         over blocks of 128 queries (causal: only those that see
 //                         the keys).  Per query block five 128 x 128 x 128 tcgen05
-//                         products, every operand in shared memory:
+//                         products:
 //                           S^T  = K Q^T           (TMEM X)
 //                           dP^T = V dO^T          (TMEM X, once S^T is read out)
-//                           dV  += P^T dO          (A = P^T bf16, smem)
-//                           dK  += dS^T Q          (A = dS^T bf16, smem, same tile)
-//                           dQ^T = K^T dS^T        (TMEM Y)
+//                           dV  += P^T dO          (A = P^T bf16 in TMEM Y)
+//                           dQ^T = K^T dS^T        (TMEM Y, after dV)
+//                           dK  += dS^T Q          (A = dS^T bf16, smem)
 //                         eight warps compute P and dS, two per SM sub-partition
 //                         (thread = key row, each warp 64 of the 128 query
-//                         columns, all of it elementwise) and write them, one
-//                         after the other, into one swizzled [key][query] tile;
+//                         columns, all of it elementwise); P goes to the low
+//                         half of Y (free once the previous dQ^T half there is
+//                         read out), dS to a swizzled [key][query] smem tile;
 //                         a warpgroup with one thread per head-dim lane drains
 //                         dQ^T into the fp32 dQ accumulator with atomic adds;
 //  * fa_bwd_dq_kernel:    dQ = bf16(scale * dQacc).
@@ -121,17 +122,17 @@ struct BwdCfg {
   static constexpr int DRAIN_THREADS = 128;
   // Register split (setmaxnreg).  448 threads launch with 128 registers each
   // (four warps share a sub-partition's 16K registers); P/dS warps take 144,
-  // the MMA and TMA warps 104, the drain warps give theirs down to 72:
-  // 256 * 144 + 128 * 72 + 64 * 104 = 52736 <= 448 * 128, and per sub-partition
-  // 2 * 144 + 72 + 104 = 464 <= 512 registers per thread slot.
+  // the MMA and TMA warps 112, the drain warps give theirs down to 80:
+  // 256 * 144 + 128 * 80 + 64 * 112 = 54272 <= 448 * 128, and per sub-partition
+  // 2 * 144 + 80 + 112 = 480 <= 512 registers per thread slot.
   static constexpr int LAUNCH_REGS = 128;
-  static constexpr int REGS_PDS = 144, REGS_DRAIN = 72, REGS_SINGLE = 104;
+  static constexpr int REGS_PDS = 144, REGS_DRAIN = 80, REGS_SINGLE = 112;
   static constexpr int REG = 128 * 128;        // one 64-column SW128 region of a 128-row bf16 tile
   static constexpr int TILE = 2 * REG;         // a 128 x 128 bf16 tile (32 KB)
   static constexpr int OFF_K = 0, OFF_V = TILE;
   static constexpr int OFF_Q = 2 * TILE;       // two Q stages
   static constexpr int OFF_DO = 4 * TILE;      // two dO stages
-  static constexpr int OFF_PS = 6 * TILE;      // P_i, then dS_i, stored [key][query]
+  static constexpr int OFF_PS = 6 * TILE;      // dS_i, stored [key][query]
   static constexpr int OFF_VEC = 7 * TILE;     // per Q stage: lse2[BM] then D[BM]
   static constexpr int VEC_BYTES = 2 * BM * 4;
   static constexpr int OFF_BAR = OFF_VEC + 2 * VEC_BYTES;
@@ -142,9 +143,10 @@ struct BwdCfg {
   // tiles) inside this and checks that USED still fits.
   static constexpr int SMEM_BYTES = 232448;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t T_DV = 0, T_DK = 128, T_X = 256, T_Y = 384;   // X: S^T, then dP^T; Y: dQ^T
+  // X: S^T, then dP^T.  Y: P^T (bf16, columns 0-63), then dQ^T (fp32, 128 columns)
+  static constexpr uint32_t T_DV = 0, T_DK = 128, T_X = 256, T_Y = 384;
   static constexpr uint32_t IDESC_SD = idesc_bf16_f32(128, BM, false, false);   // S^T, dP^T
-  static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);     // dV, dK
+  static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);     // dV (A in TMEM), dK
   static constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, BM, true, true);      // dQ^T
 };
 static_assert(BwdCfg::USED + 768 <= BwdCfg::SMEM_BYTES, "shared memory plan");
@@ -197,12 +199,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const uint32_t b_s_full = bar(9);      // S_i in X
   const uint32_t b_dp_full = bar(10);    // dP_i in X
   const uint32_t b_x_free = bar(11);     // X read out (twice per query block: S, then dP)
-  const uint32_t b_p_ready = bar(12);    // P_i in the P/dS tile
-  const uint32_t b_dv_done = bar(13);    // dV_i done reading P_i
-  const uint32_t b_ds_ready = bar(14);   // dS_i in the P/dS tile
-  const uint32_t b_ps_free = bar(15);    // dK_i, dQ_i done reading dS_i
+  const uint32_t b_p_ready = bar(12);    // P_i in the low half of Y
+  const uint32_t b_ylo_free = bar(13);   // low half of Y read out (dQ^T_i, queries 0-63)
+  const uint32_t b_ds_ready = bar(14);   // dS_i in the dS tile
+  const uint32_t b_ps_free = bar(15);    // dQ_i, dK_i done reading dS_i
   const uint32_t b_dq_full = bar(16);    // dQ^T_i in Y
-  const uint32_t b_dq_free = bar(17);    // Y read out
+  const uint32_t b_yhi_free = bar(17);   // all of Y read out
   const uint32_t b_dkv_done = bar(18);
   const uint32_t b_drain = bar(19);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -229,11 +231,11 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     mbar_init(b_dp_full, 1);
     mbar_init(b_x_free, C::PDS_THREADS);
     mbar_init(b_p_ready, C::PDS_THREADS);
-    mbar_init(b_dv_done, 1);
+    mbar_init(b_ylo_free, C::DRAIN_THREADS);
     mbar_init(b_ds_ready, C::PDS_THREADS);
     mbar_init(b_ps_free, 1);
     mbar_init(b_dq_full, 1);
-    mbar_init(b_dq_free, C::DRAIN_THREADS);
+    mbar_init(b_yhi_free, C::DRAIN_THREADS);
     mbar_init(b_dkv_done, 1);
     mbar_init(b_drain, 1);
     fence_mbar_init();
@@ -253,7 +255,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   if (warp == 13) {
     // ------------------------------------------------------------ TMA producer
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 112;");
     if (lane == 0) {
       bool ok = true;
       int q_last[2] = {-1, -1}, do_last[2] = {-1, -1};     // last query block loaded into each stage
@@ -290,7 +292,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 112;");
     if (lane == 0) {
       // Descriptors are built once; a K step adds to the start-address field:
       // K-major tiles advance 32 B inside a 128-B row and switch region every
@@ -309,11 +311,17 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) umma_ss(tmem + C::T_X, a + kstep(kk), b + kstep(kk), C::IDESC_SD, kk > 0);
       };
-      // dV += P^T dO, dK += dS^T Q: A = the P/dS tile (K-major), B MN-major
-      auto issue_kv = [&](uint32_t d_tmem, uint64_t b, bool acc) {
+      // dV += P^T dO (A = P^T in Y, 8 packed columns per K step), dK += dS^T Q
+      // (A = the dS tile, K-major); B MN-major
+      auto issue_dv = [&](uint64_t b, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < C::BM / 16; ++kk)
-          umma_ss(d_tmem, dPS_k + kstep(kk), b + mnstep(kk), C::IDESC_KV, (acc || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + C::T_DV, tmem + C::T_Y + 8 * kk, b + mnstep(kk), C::IDESC_KV, (acc || kk > 0) ? 1u : 0u);
+      };
+      auto issue_dk = [&](uint64_t b, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < C::BM / 16; ++kk)
+          umma_ss(tmem + C::T_DK, dPS_k + kstep(kk), b + mnstep(kk), C::IDESC_KV, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(b_kv_full, 0, ctl);
       // prologue: S_0, and dP_0 once S_0 has been read out of X
@@ -337,8 +345,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // dV += P_i^T dO_i
         if (!mbar_wait(b_p_ready, ph, ctl)) { ok = false; break; }
         tc_fence_after();
-        issue_kv(tmem + C::T_DV, s ? dO_mn1 : dO_mn0, it > 0);
-        umma_commit(b_dv_done);
+        issue_dv(s ? dO_mn1 : dO_mn0, it > 0);
         umma_commit(b_do_empty(s));
         // S_{i+1}, once dP_i has been read out of X
         if (more) {
@@ -347,19 +354,16 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           issue_kmaj(dK_k, s ? dQ_k0 : dQ_k1);
           umma_commit(b_s_full);
         }
-        // dK += dS_i^T Q_i, dQ^T_i = K^T dS_i^T
+        // dQ^T_i = K^T dS_i^T (into Y, after dV_i has read P_i there), then dK += dS_i^T Q_i
         if (!mbar_wait(b_ds_ready, ph, ctl)) { ok = false; break; }
+        if (it > 0 && !mbar_wait(b_yhi_free, ph ^ 1u, ctl)) { ok = false; break; }
         tc_fence_after();
-        issue_kv(tmem + C::T_DK, s ? dQ_mn1 : dQ_mn0, it > 0);
-        umma_commit(b_q_empty(s));
-        if (it > 0) {
-          if (!mbar_wait(b_dq_free, ph ^ 1u, ctl)) { ok = false; break; }
-          tc_fence_after();
-        }
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
           umma_ss(tmem + C::T_Y, dK_mn + mnstep(kk), dPS_mn + mnstep(kk), C::IDESC_Q, kk > 0);
         umma_commit(b_dq_full);
+        issue_dk(s ? dQ_mn1 : dQ_mn0, it > 0);
+        umma_commit(b_q_empty(s));
         umma_commit(b_ps_free);
         // dP_{i+1}, once S_{i+1} has been read out of X
         if (more) {
@@ -382,9 +386,10 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int key = k0 + rloc;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tX = tmem + lane_off + C::T_X + 64 * ch;
+    const uint32_t tP = tmem + lane_off + C::T_Y + 32 * ch;     // this thread's 64 P values, packed
     const float c2 = args.scale_log2;
     const bool key_ok = key < args.N;
-    // this thread's half row of the P / dS tile: region ch, row rloc; 16-byte
+    // this thread's half row of the dS tile: region ch, row rloc; 16-byte
     // chunk j of the row sits at chunk j ^ (row & 7) (128-byte swizzle)
     uint8_t* prow = smem + C::OFF_PS + ch * C::REG + rloc * 128;
     const int sw = rloc & 7;
@@ -408,6 +413,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         reg_fence32(rb);
         tc_fence_before();
         mbar_arrive(b_x_free);
+        // 2^x: three pairs in eight on the FMA pipe (ex2_poly2), the rest on the
+        // special-function unit, which would otherwise be the limit here
         const float2 c2v = make_float2(c2, c2);
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
@@ -417,10 +424,18 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                   make_float2(-la.x, -la.y));
           const float2 xb = ffma2(make_float2(__uint_as_float(rb[c]), __uint_as_float(rb[c + 1])), c2v,
                                   make_float2(-lb.x, -lb.y));
-          p[c] = ex2_approx(xa.x);
-          p[c + 1] = ex2_approx(xa.y);
-          p[32 + c] = ex2_approx(xb.x);
-          p[32 + c + 1] = ex2_approx(xb.y);
+          if ((0x92u >> ((c >> 1) & 7)) & 1u) {
+            const float2 ea = ex2_poly2(xa), eb = ex2_poly2(xb);
+            p[c] = ea.x;
+            p[c + 1] = ea.y;
+            p[32 + c] = eb.x;
+            p[32 + c + 1] = eb.y;
+          } else {
+            p[c] = ex2_approx(xa.x);
+            p[c + 1] = ex2_approx(xa.y);
+            p[32 + c] = ex2_approx(xb.x);
+            p[32 + c + 1] = ex2_approx(xb.y);
+          }
         }
       }
       // keys past the sequence end, and (causal) queries before this key, get P = 0
@@ -433,11 +448,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-      if (it > 0 && !mbar_wait_warp(b_ps_free, ph ^ 1u, ctl)) { ok = false; break; }
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4*>(prow + ((j ^ sw) << 4)) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-      fence_proxy_async_smem();
+      // P^T into the low half of Y, once the previous dQ^T there has been read out
+      if (it > 0 && !mbar_wait_warp(b_ylo_free, ph ^ 1u, ctl)) { ok = false; break; }
+      tc_fence_after();
+      tmem_st32(tP, pk);
+      tmem_wait_st();
+      tc_fence_before();
       mbar_arrive(b_p_ready);
       // dS = P (dP - D)
       if (!mbar_wait_warp(b_dp_full, ph, ctl)) { ok = false; break; }
@@ -460,7 +476,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           pk[16 * h + (c >> 1)] = pack_bf16x2(g.x, g.y);
         }
       }
-      if (!mbar_wait_warp(b_dv_done, ph, ctl)) { ok = false; break; }
+      if (it > 0 && !mbar_wait_warp(b_ps_free, ph ^ 1u, ctl)) { ok = false; break; }
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         *reinterpret_cast<uint4*>(prow + ((j ^ sw) << 4)) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
@@ -499,7 +515,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
   } else {
     // ------------------------------------------------------------ dQ drain (thread = head-dim lane)
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
     const int dl = (warp - 8) * 32 + lane;
     const uint32_t tY = tmem + (static_cast<uint32_t>((warp - 8) * 32) << 16) + C::T_Y;
     float* acc = args.dq_acc + static_cast<size_t>(bh) * args.N * D + dl;
@@ -509,17 +525,15 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const int q0 = (i_begin + it) * C::BM;
       const int nq = min(C::BM, args.N - q0);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {      // two 64-column halves (register budget); Y is free after the second load
+      for (int h = 0; h < 2; ++h) {      // two 64-column halves (register budget), each released once loaded
         uint32_t r[64];
         tmem_ld32(tY + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(r));
         tmem_ld32(tY + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
         tmem_wait_ld();
         reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r));
         reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r + 32));
-        if (h == 1) {
-          tc_fence_before();
-          mbar_arrive(b_dq_free);
-        }
+        tc_fence_before();
+        mbar_arrive(h == 0 ? b_ylo_free : b_yhi_free);
         float* a_row = acc + static_cast<size_t>(q0 + 64 * h) * D;
         const int nh = nq - 64 * h;      // valid rows in this half (may be <= 0)
         if (nh >= 64) {
