@@ -51,7 +51,7 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-heads", type=int, default=2, help="heads in the CPU baseline sample")
+    p.add_argument("--cpu-heads", type=int, default=6, help="heads in the CPU baseline sample")
     p.add_argument("--shape", default=None,
                    help="B,H,N override of the workload's sizes (smaller cases for profiler captures)")
     return p.parse_args()
