@@ -36,6 +36,9 @@ from exact_io_aware_100_b200 import inputs  # noqa: E402
 METRIC = "attention fwd/bwd TFLOP/s (bf16, causal & non-causal); % of B200 BF16 peak"
 DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2**20
+EX2_PER_CLK_PER_SM = 16      # MUFU ex2 rate measured on this GPU by a probe (16 lanes / clock / SM)
+MUFU_SHARE_OF_EXP = 5 / 8    # both kernels evaluate three of every eight exp2 pairs by polynomial
 KERNEL_SOURCES = ["exact_io_aware_100_b200/csrc/ptx.cuh", "exact_io_aware_100_b200/csrc/fwd_kernel.cuh",
                   "exact_io_aware_100_b200/csrc/bwd_kernel.cuh"]
 
@@ -266,11 +269,19 @@ def main():
     shape = (B, H, N, d)
     seed = w.seed + 100003 * rank          # each rank its own batch
     names = ("q", "k", "v") if fwd_only else ("q", "k", "v", "do")
-    host = {n: inputs.make_tensor(seed, n, shape, w.k_scale if n == "k" else 1.0, "bf16") for n in names}
-    pinned = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in names}
+    f32_in = w.dtype == "f32"               # fp32 inputs go through fa_fwd_ex (cast to bf16 on the GPU)
+    host = {n: inputs.make_tensor(seed, n, shape, w.k_scale if n == "k" else 1.0, "f32" if f32_in else "bf16")
+            for n in names}
+    if f32_in:
+        pinned = {n: torch.from_numpy(host[n]).pin_memory() for n in names}
+    else:
+        pinned = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in names}
     dv_ = {n: pinned[n].to(dev) for n in names}
-    o = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    o = torch.empty(shape, dtype=torch.float32 if f32_in else torch.bfloat16, device=dev)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    fws = None
+    if f32_in:
+        fws = torch.empty(fa.fa_fwd_workspace_size(B, H, N, d, fa.FA_F32), dtype=torch.uint8, device=dev)
     if not fwd_only:
         dq, dk, dvv = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
         ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
@@ -280,7 +291,10 @@ def main():
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        fa.fa_fwd(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, stream=stream)
+        if f32_in:
+            fa.fa_fwd_ex(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, fa.FA_F32, fws, stream=stream)
+        else:
+            fa.fa_fwd(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, stream=stream)
         if ev is not None:
             ev[1].record(stream)
         if fwd_only:
@@ -295,7 +309,14 @@ def main():
         if ev is not None:
             ev[4].record(stream)
 
-    launches_per_step = 1 if fwd_only else 4
+    launches_per_step = (4 if f32_in else 1) if fwd_only else 4    # fp32: three cast kernels + the forward
+    # Inputs and outputs smaller than twice L2 would stay cached between steps:
+    # then every timed step is preceded by a write of a buffer larger than L2,
+    # outside the kernels' events, and the step time is the sum of its events.
+    io_bytes = sum(host[n].nbytes for n in names) * (2 if not fwd_only else 1) + o.numel() * o.element_size()
+    flush = None
+    if io_bytes < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -310,15 +331,21 @@ def main():
     with ClockSampler(local_rank) as clk:
         t0.record(stream)
         for s in range(args.steps):
+            if flush is not None:
+                flush.fill_(s & 0xff)
             step(evs[s])
         t1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
+    last = 1 if fwd_only else 4
+    step_ms = [e[0].elapsed_time(e[last]) for e in evs]
+    elapsed_ms = sum(step_ms) if flush is not None else t0.elapsed_time(t1)
     if fa.fa_get_device_status() != fa.FA_OK:
         raise SystemExit("device status reported a timeout in the timed region")
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    fwd_all = [e[0].elapsed_time(e[1]) for e in evs]
+    main_all = None if fwd_only else [e[2].elapsed_time(e[3]) for e in evs]
+    fwd_ms = statistics.mean(fwd_all)
     main_ms = None if fwd_only else statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     prep_ms = None if fwd_only else statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     fin_ms = None if fwd_only else statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
@@ -334,12 +361,19 @@ def main():
     peaks, peak_src = load_peaks()
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
 
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     fwd_tf = fwd_flops / (fwd_ms * 1e-3) / 1e12
-    kernels = {"fa_fwd_kernel": {"ms": fwd_ms, "tflops": fwd_tf, "frac_of_measured_burst": fwd_tf / burst,
+    kernels = {"fa_fwd_kernel": {"ms": fwd_ms, "median_ms": statistics.median(fwd_all), "min_ms": min(fwd_all),
+                                 "tflops": fwd_tf, "frac_of_measured_burst": fwd_tf / burst,
+                                 "frac_of_measured_sustained": fwd_tf / sustained,
                                  "frac_of_datasheet": fwd_tf / DATASHEET_BF16_TFLOPS}}
+    if f32_in:
+        kernels["fa_fwd_kernel"]["note"] = "fa_fwd_ex(FA_F32): three cast kernels + the forward"
     if not fwd_only:
         main_tf = bwd_flops / (main_ms * 1e-3) / 1e12
-        kernels["fa_bwd_kernel"] = {"ms": main_ms, "tflops": main_tf, "frac_of_measured_burst": main_tf / burst,
+        kernels["fa_bwd_kernel"] = {"ms": main_ms, "median_ms": statistics.median(main_all), "min_ms": min(main_all),
+                                    "tflops": main_tf, "frac_of_measured_burst": main_tf / burst,
+                                    "frac_of_measured_sustained": main_tf / sustained,
                                     "frac_of_datasheet": main_tf / DATASHEET_BF16_TFLOPS}
         kernels["fa_bwd_pre_kernel"] = {"ms": prep_ms}
         kernels["fa_bwd_dq_kernel"] = {"ms": fin_ms}
@@ -348,7 +382,16 @@ def main():
     achieved = kernels[dom]["tflops"]
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
                 "frac": achieved / burst, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "frac_of_sustained": achieved / sustained,
                 "flops_per_launch": dom_flops, "traffic": committed_traffic(dom, w.name)}
+    # forward HBM: each input read once, O and lse written once (the IO-aware minimum)
+    in_elem = 4 if f32_in else 2
+    fwd_bytes = B * H * N * d * (3 * in_elem + o.element_size()) + 4 * B * H * N
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fwd_hbm = {"algorithmic_bytes": fwd_bytes, "gbs": fwd_bytes / (fwd_ms * 1e-3) / 1e9,
+               "frac_of_measured_hbm": fwd_bytes / (fwd_ms * 1e-3) / 1e9 / hbm}
+    # exponentials: one per visible score in the forward, recomputed once in the backward
+    n_exp = B * H * (N * (N + 1) // 2 if causal else N * N)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
     e2e = None
@@ -396,13 +439,23 @@ def main():
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(w, "fwd" if fwd_only else "fwd+bwd",
-                                  f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB per step), no flush"),
+                                  f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB per step), no flush"
+                                  if flush is None else
+                                  f"L2 flushed before every step ({2 * L2_BYTES / 2**20:.0f} MiB write, outside the "
+                                  f"kernel events; value from the summed step events)"),
         "frac_of_measured_burst_peak": value / world / burst,
         "frac_of_datasheet_peak": value / world / DATASHEET_BF16_TFLOPS,
         "fwd_tflops": fwd_tf, "bwd_tflops": None if fwd_only else bwd_flops / ((prep_ms + main_ms + fin_ms) * 1e-3) / 1e12,
         "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(),
+        "fwd_hbm": fwd_hbm,
     }
+    sm_mhz = line["clocks"].get("sm_mhz") or 1965.0
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    mufu_s = n_exp * MUFU_SHARE_OF_EXP / (EX2_PER_CLK_PER_SM * n_sm * sm_mhz * 1e6)
+    line["exp"] = {"count_fwd": n_exp, "count_bwd": 0 if fwd_only else n_exp, "on_mufu": MUFU_SHARE_OF_EXP,
+                   "mufu_time_share_fwd": mufu_s / (fwd_ms * 1e-3),
+                   "mufu_time_share_bwd": None if fwd_only else mufu_s / (main_ms * 1e-3)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
