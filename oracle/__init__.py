@@ -2,7 +2,9 @@
 from .attention import (  # noqa: F401
     as_f64,
     attention_bwd,
+    attention_bwd_gqa,
     attention_fwd,
+    attention_fwd_gqa,
     attention_fwd_blockwise,
     attention_fwd_rows,
     softmax_merge,

@@ -19,7 +19,10 @@ Sources (the pages this follows; cited by title and section):
      section "تکنیک 2: محاسبه مجدد" (the backward recomputes the attention
      matrix instead of storing it).
 [P3] nearauto.com FlashAttention-2 digest, section on reducing non-matmul
-     FLOPs (normalise once, outputs unchanged).
+     FLOPs (normalise once, outputs unchanged), and section
+     "新機能: 最大256のヘッドディメンション、マルチクエリアテンション" (multi-query and
+     grouped-query attention: one key/value head shared by a set of query
+     heads); the unite.ai page lists the same variants under "FlashAttention-2".
 
 Every function here is the plain definition written out in float64 with numpy:
 the score matrix S and the probabilities P are materialised for whole rows,
@@ -37,7 +40,11 @@ Readings where the pages are silent or garbled (each is listed in the design doc):
   * the garbled merge formula is read as l = e^(m_x-m) l_x + e^(m_y-m) l_y and
     softmax(x u y) = [e^(m_x-m) l_x softmax(x), e^(m_y-m) l_y softmax(y)] / l;
   * the backward is the exact gradient of the forward (the pages only say
-    "recompute"), with D_i = sum_j P_ij dP_ij.
+    "recompute"), with D_i = sum_j P_ij dP_ij;
+  * grouped-query attention: the pages say each set of query heads shares one
+    key/value head but not which; the sets are contiguous, query head h using
+    key/value head h // (H / H_kv), and a shared head's gradient is the sum of
+    the gradients of its uses.
 
 Parity pins for every function live in tests/test_oracle.py; none of the
 functions below is "parity unpinned".
@@ -51,6 +58,8 @@ __all__ = [
     "attention_fwd",
     "attention_fwd_rows",
     "attention_bwd",
+    "attention_fwd_gqa",
+    "attention_bwd_gqa",
     "softmax_merge",
     "attention_fwd_blockwise",
 ]
@@ -154,6 +163,55 @@ def attention_bwd(q, k, v, do, scale: float, causal: bool):
             ds = p * (dp - dd)
             dq[b, h] = scale * (ds @ k[b, h])
             dk[b, h] = scale * (ds.T @ q[b, h])
+    return dq, dk, dv
+
+
+def _kv_head(h: int, H: int, H_kv: int) -> int:
+    """Key/value head read by query head h: contiguous sets of H / H_kv query heads."""
+    if H_kv < 1 or H % H_kv != 0:
+        raise ValueError("the query head count must be a multiple of the key/value head count")
+    return h // (H // H_kv)
+
+
+def attention_fwd_gqa(q, k, v, scale: float, causal: bool):
+    """Grouped-query (and multi-query, H_kv = 1) forward.
+
+    [P3] "新機能: 最大256のヘッドディメンション、マルチクエリアテンション": a set of
+    query heads shares one key/value head.  q is [B, H, N, d]; k, v are
+    [B, H_kv, N, d] with H a multiple of H_kv.  Each query head is exactly the
+    ``attention_fwd`` of its own queries against its set's keys and values.
+    Returns (O [B,H,N,d_v], lse [B,H,N]) in float64.
+    """
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    B, H, N, _ = q.shape
+    H_kv = k.shape[1]
+    o = np.empty((B, H, N, v.shape[-1]), dtype=np.float64)
+    lse = np.empty((B, H, N), dtype=np.float64)
+    for h in range(H):
+        g = _kv_head(h, H, H_kv)
+        o_h, lse_h = attention_fwd(q[:, h:h + 1], k[:, g:g + 1], v[:, g:g + 1], scale, causal)
+        o[:, h], lse[:, h] = o_h[:, 0], lse_h[:, 0]
+    return o, lse
+
+
+def attention_bwd_gqa(q, k, v, do, scale: float, causal: bool):
+    """Exact gradients of sum(dO * O) for O = attention_fwd_gqa(...).
+
+    dQ of a query head is that head's ``attention_bwd`` dQ; a key/value head is
+    an input of every query head in its set, so its dK and dV are the sums of
+    those heads' dK and dV.  Returns float64 arrays shaped like q, k, v.
+    """
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    B, H, N, _ = q.shape
+    H_kv = k.shape[1]
+    dq = np.empty_like(q)
+    dk, dv = np.zeros_like(k), np.zeros_like(v)
+    for h in range(H):
+        g = _kv_head(h, H, H_kv)
+        dq_h, dk_h, dv_h = attention_bwd(q[:, h:h + 1], k[:, g:g + 1], v[:, g:g + 1], do[:, h:h + 1], scale, causal)
+        dq[:, h] = dq_h[:, 0]
+        dk[:, g] += dk_h[:, 0]
+        dv[:, g] += dv_h[:, 0]
     return dq, dk, dv
 
 

@@ -13,8 +13,8 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (attention_bwd, attention_fwd, attention_fwd_blockwise,
-                    attention_fwd_rows, softmax_merge)
+from oracle import (attention_bwd, attention_bwd_gqa, attention_fwd, attention_fwd_blockwise,
+                    attention_fwd_gqa, attention_fwd_rows, softmax_merge)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
@@ -246,6 +246,84 @@ def test_gradient_sums():
         dq, dk, dv = attention_bwd(q, k, v, do, 0.3, causal)
         np.testing.assert_allclose(dv.sum(2), do.sum(2), atol=1e-12)
         np.testing.assert_allclose(dk.sum(2), 0.0, atol=1e-12)
+
+
+# --- grouped-query attention ---------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_matches_torch_sdpa_enable_gqa(causal):
+    """torch's scaled-dot-product attention with enable_gqa (CPU, float64), forward and autograd:
+    an independent implementation of contiguous query-head sets sharing a key/value head."""
+    B, H, H_kv, N, d, scale = 2, 6, 2, 41, 8, 0.3
+    q, do = _rand((B, H, N, d), 81), _rand((B, H, N, d), 82)
+    k, v = _rand((B, H_kv, N, d), 83), _rand((B, H_kv, N, d), 84)
+    o, lse = attention_fwd_gqa(q, k, v, scale, causal)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale,
+                                                          enable_gqa=True)
+    np.testing.assert_allclose(o, to.detach().numpy(), atol=1e-12)
+    to.backward(torch.tensor(do))
+    dq, dk, dv = attention_bwd_gqa(q, k, v, do, scale, causal)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-11)
+    # lse of query head h equals the plain forward's lse against key/value head h // 3
+    _, lse1 = attention_fwd(q[:, 4:5], k[:, 1:2], v[:, 1:2], scale, causal)
+    np.testing.assert_allclose(lse[:, 4], lse1[:, 0], atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_gradients_by_central_differences(causal):
+    """Brute force on a tiny case: the shared key/value heads' gradients sum over their sets."""
+    H, H_kv, N, d, scale, h = 4, 2, 5, 3, 0.7, 1e-6
+    q, do = _rand((1, H, N, d), 91), _rand((1, H, N, d), 92)
+    k, v = _rand((1, H_kv, N, d), 93), _rand((1, H_kv, N, d), 94)
+    grads = attention_bwd_gqa(q, k, v, do, scale, causal)
+
+    def loss(qq, kk, vv):
+        o, _ = attention_fwd_gqa(qq, kk, vv, scale, causal)
+        return float((o * do).sum())
+
+    for which, grad in enumerate(grads):
+        fd = np.zeros_like(grad)
+        for idx in np.ndindex(grad.shape):
+            args = [q.copy(), k.copy(), v.copy()]
+            args[which][idx] += h
+            lp = loss(*args)
+            args[which][idx] -= 2 * h
+            lm = loss(*args)
+            fd[idx] = (lp - lm) / (2 * h)
+        rel = np.abs(fd - grad).max() / max(np.abs(grad).max(), 1e-30)
+        assert rel < 1e-6, (which, rel)
+
+
+def test_gqa_special_cases():
+    """H_kv = H is plain multi-head attention; identical query heads over one shared
+    key/value head (multi-query) give identical outputs and H times one head's dK, dV."""
+    q, k, v, do = (_rand((2, 3, 19, 8), 100 + i) for i in range(4))
+    for causal in (False, True):
+        o, lse = attention_fwd_gqa(q, k, v, 0.4, causal)
+        o1, lse1 = attention_fwd(q, k, v, 0.4, causal)
+        np.testing.assert_allclose(o, o1, atol=1e-14)
+        np.testing.assert_allclose(lse, lse1, atol=1e-14)
+        for a, b in zip(attention_bwd_gqa(q, k, v, do, 0.4, causal), attention_bwd(q, k, v, do, 0.4, causal)):
+            np.testing.assert_allclose(a, b, atol=1e-14)
+    q1, do1 = _rand((1, 1, 23, 8), 110), _rand((1, 1, 23, 8), 111)
+    k1, v1 = _rand((1, 1, 23, 8), 112), _rand((1, 1, 23, 8), 113)
+    H = 4
+    qh, doh = np.repeat(q1, H, axis=1), np.repeat(do1, H, axis=1)
+    o, _ = attention_fwd_gqa(qh, k1, v1, 0.5, True)
+    for hh in range(H):
+        np.testing.assert_allclose(o[:, hh], o[:, 0], atol=1e-15)
+    _, dk, dv = attention_bwd_gqa(qh, k1, v1, doh, 0.5, True)
+    _, dk1, dv1 = attention_bwd(q1, k1, v1, do1, 0.5, True)
+    np.testing.assert_allclose(dk, H * dk1, atol=1e-12)
+    np.testing.assert_allclose(dv, H * dv1, atol=1e-12)
+
+
+def test_gqa_rejects_uneven_sets():
+    with pytest.raises(ValueError):
+        attention_fwd_gqa(_rand((1, 3, 4, 2), 1), _rand((1, 2, 4, 2), 2), _rand((1, 2, 4, 2), 3), 1.0, False)
 
 
 # --- the softmax merge and the blockwise algorithm -------------------------
