@@ -23,7 +23,7 @@ FA_BF16, FA_F32 = 0, 1
 
 EXPORTS = (
     "fa_fwd", "fa_fwd_ex", "fa_fwd_workspace_size", "fa_bwd", "fa_bwd_workspace_size",
-    "fa_bwd_prepare", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc",
+    "fa_bwd_prepare", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc", "fa_fwd_gqa", "fa_bwd_gqa",
     "fa_get_device_status", "fa_selftest_wait_timeout", "fa_status_string", "fa_version",
 )
 
@@ -55,6 +55,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_bwd_main.argtypes = [P, P, P, P, P, P, I, I, I, I, F, I, P, Z, P]
     L.fa_bwd_finish.argtypes = [P, I, I, I, I, F, P, Z, P]
     L.fa_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P]
+    L.fa_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P]
+    L.fa_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, Z, P]
     L.fa_bwd_workspace_size.argtypes = [I, I, I, I]
     L.fa_bwd_workspace_size.restype = Z
     L.fa_get_device_status.argtypes = [P]
@@ -63,7 +65,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_version.restype = ctypes.c_char_p
     for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_prepare", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc",
-                 "fa_get_device_status", "fa_selftest_wait_timeout"):
+                 "fa_fwd_gqa", "fa_bwd_gqa", "fa_get_device_status", "fa_selftest_wait_timeout"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -176,6 +178,26 @@ def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float
                                          _stream(stream)), "fa_bwd_noalloc")
 
 
+def fa_fwd_gqa(q, k, v, o, lse, causal: bool, scale: float | None = None, stream=None) -> None:
+    """Grouped-query forward: q, o [B,H,N,d]; k, v [B,H_kv,N,d] (H a multiple of H_kv)."""
+    B, H, N, d = _bhnd(q)
+    H_kv = _bhnd(k)[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(load_library().fa_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, H_kv, N, d, scale,
+                                     int(bool(causal)), _stream(stream)), "fa_fwd_gqa")
+
+
+def fa_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, workspace, scale: float | None = None,
+               stream=None) -> None:
+    """Grouped-query backward: dk, dv [B,H_kv,N,d] are sums over each key/value head's query set."""
+    B, H, N, d = _bhnd(q)
+    H_kv = _bhnd(k)[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(load_library().fa_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                                     _ptr(dk), _ptr(dv), B, H, H_kv, N, d, scale, int(bool(causal)),
+                                     _ptr(workspace), _ws_bytes(workspace), _stream(stream)), "fa_bwd_gqa")
+
+
 def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
     return int(load_library().fa_bwd_workspace_size(B, H, N, d))
 
@@ -198,12 +220,15 @@ def _workspace(nbytes: int, device):
 
 
 def forward(q, k, v, causal: bool, scale: float | None = None, stream=None):
-    """O, lse for [B,H,N,d] tensors (bf16, or float32 via the bf16 tensor-core path)."""
+    """O, lse for q [B,H,N,d] and k, v [B,H_kv,N,d] (bf16; float32 via the bf16 tensor-core path when
+    H_kv == H).  H_kv < H is grouped-query attention (contiguous sets of H / H_kv query heads)."""
     import torch
     B, H, N, d = _bhnd(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if q.dtype == torch.bfloat16:
+    if _bhnd(k)[1] != H:          # fewer key/value heads: grouped-query attention
+        fa_fwd_gqa(q, k, v, o, lse, causal, scale, stream)
+    elif q.dtype == torch.bfloat16:
         fa_fwd(q, k, v, o, lse, causal, scale, stream)
     elif q.dtype == torch.float32:
         ws = _workspace(fa_fwd_workspace_size(B, H, N, d, FA_F32), q.device)
@@ -214,11 +239,15 @@ def forward(q, k, v, causal: bool, scale: float | None = None, stream=None):
 
 
 def backward(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, stream=None, workspace=None):
-    """dQ, dK, dV (bf16) from the forward's O and lse."""
+    """dQ, dK, dV (bf16) from the forward's O and lse; dK, dV have k's head count (grouped-query
+    attention sums each shared head's gradient over its set)."""
     import torch
     B, H, N, d = _bhnd(q)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
         workspace = _workspace(fa_bwd_workspace_size(B, H, N, d), q.device)
-    fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal, workspace, scale, stream)
+    if _bhnd(k)[1] != H:
+        fa_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, causal, workspace, scale, stream)
+    else:
+        fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal, workspace, scale, stream)
     return dq, dk, dv

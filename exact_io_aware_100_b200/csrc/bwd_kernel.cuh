@@ -12,9 +12,12 @@
 //
 // Kernels:
 //  * fa_bwd_pre_kernel:   D_i, lse_i * log2(e) (padded rows get +inf), dQacc = 0
-//  * fa_bwd_kernel:       one CTA per (batch*head, block of 128 keys), looping
-//                         over blocks of 128 queries (causal: only those that see
-//                         the keys).  Per query block five 128 x 128 x 128 tcgen05
+//  * fa_bwd_kernel:       one CTA per (batch * key/value head, block of 128
+//                         keys), looping over blocks of 128 queries (causal: only
+//                         those that see the keys) of every query head that reads
+//                         this key/value head (one for multi-head attention, a
+//                         set of consecutive heads for grouped-query attention, so
+//                         dK and dV of the shared head sum over the set in TMEM).  Per query block five 128 x 128 x 128 tcgen05
 //                         products:
 //                           S^T  = K Q^T           (TMEM X)
 //                           dP^T = V dO^T          (TMEM X, once S^T is read out)
@@ -46,7 +49,10 @@ struct BwdArgs {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   uint32_t* status;
-  int N, Np, bh;          // Np = n_qb * 128
+  int N, Np, bh;          // Np = n_qb * 128; bh = B * H (query heads)
+  int bh_kv;              // B * H_kv (key/value heads); the main kernel's work items
+  int heads;              // H
+  int group;              // query heads per key/value head
   int n_kb;               // ceil(N / 128) key blocks
   int n_qb;               // ceil(N / 128) query blocks
   int heads_per_group;    // work-item order of the main kernel
@@ -165,7 +171,7 @@ __device__ __forceinline__ void bwd_decode(const BwdArgs& a, int x, int& bh, int
   const int g = x / per_group;
   const int r = x - g * per_group;
   const int h0 = g * a.heads_per_group;
-  const int gh = min(a.heads_per_group, a.bh - h0);
+  const int gh = min(a.heads_per_group, a.bh_kv - h0);
   kb = r / gh;
   bh = h0 + (r - kb * gh);
 }
@@ -212,11 +218,17 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  int bh, kb;
+  int bh, kb;                                        // bh: key/value head
   bwd_decode(args, static_cast<int>(blockIdx.x), bh, kb);
   const int k0 = kb * C::BN;
   const int i_begin = args.causal ? kb : 0;          // query blocks that see these keys (BM == BN)
-  const int n_iter = args.n_qb - i_begin;
+  const int n_per = args.n_qb - i_begin;             // per query head
+  const int n_iter = n_per * args.group;             // every query head of the set, one after the other
+  // query head and query block of iteration it
+  const int h_kv_count = args.heads / args.group;
+  const int bhq0 = (bh / h_kv_count) * args.heads + (bh % h_kv_count) * args.group;
+  auto q_head = [&](int it) { return bhq0 + it / n_per; };
+  auto q_row0 = [&](int it) { return (i_begin + it % n_per) * C::BM; };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0u;
@@ -267,19 +279,20 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       for (int it = 0; it < n_iter; ++it) {
         const int s = it & 1;
         const uint32_t round = static_cast<uint32_t>(it) >> 1;
-        const int q0 = (i_begin + it) * C::BM;
+        const int q0 = q_row0(it);
+        const int hq = q_head(it);
         // Q_i with its lse2 and D rows; the stage is released after dK_i
         if (round > 0 && !mbar_wait(b_q_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
         mbar_expect_tx(b_q_full(s), C::TILE + C::VEC_BYTES);
-        for (int r = 0; r < 2; ++r) tma_load_3d(sQ(s) + r * C::REG, &tm_q, b_q_full(s), r * 64, q0, bh);
-        const size_t voff = static_cast<size_t>(bh) * args.Np + q0;
+        for (int r = 0; r < 2; ++r) tma_load_3d(sQ(s) + r * C::REG, &tm_q, b_q_full(s), r * 64, q0, hq);
+        const size_t voff = static_cast<size_t>(hq) * args.Np + q0;
         bulk_load(sVec(s), args.lse2 + voff, C::BM * 4, b_q_full(s));
         bulk_load(sVec(s) + C::BM * 4, args.dvec + voff, C::BM * 4, b_q_full(s));
         q_last[s] = it;
         // dO_i; the stage is released after dV_i
         if (round > 0 && !mbar_wait(b_do_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
         mbar_expect_tx(b_do_full(s), C::TILE);
-        for (int r = 0; r < 2; ++r) tma_load_3d(sDO(s) + r * C::REG, &tm_do, b_do_full(s), r * 64, q0, bh);
+        for (int r = 0; r < 2; ++r) tma_load_3d(sDO(s) + r * C::REG, &tm_do, b_do_full(s), r * 64, q0, hq);
         do_last[s] = it;
       }
       if (!ok) {       // let the loads in flight land before the CTA exits
@@ -397,7 +410,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     for (int it = 0; it < n_iter; ++it) {
       const int s = it & 1;
       const uint32_t ph = static_cast<uint32_t>(it) & 1;
-      const int q0 = (i_begin + it) * C::BM;
+      const int q0 = q_row0(it);
       const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * C::VEC_BYTES) + 64 * ch;
       const float* dvec = lse2 + C::BM;
       if (!mbar_wait_warp(b_q_full(s), (static_cast<uint32_t>(it) >> 1) & 1, ctl)) { ok = false; break; }
@@ -518,11 +531,11 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
     const int dl = (warp - 8) * 32 + lane;
     const uint32_t tY = tmem + (static_cast<uint32_t>((warp - 8) * 32) << 16) + C::T_Y;
-    float* acc = args.dq_acc + static_cast<size_t>(bh) * args.N * D + dl;
     for (int it = 0; it < n_iter; ++it) {
       if (!mbar_wait_warp(b_dq_full, static_cast<uint32_t>(it) & 1, ctl)) break;
       tc_fence_after();
-      const int q0 = (i_begin + it) * C::BM;
+      const int q0 = q_row0(it);
+      float* acc = args.dq_acc + static_cast<size_t>(q_head(it)) * args.N * D + dl;
       const int nq = min(C::BM, args.N - q0);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {      // two 64-column halves (register budget), each released once loaded

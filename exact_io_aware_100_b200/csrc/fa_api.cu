@@ -126,7 +126,8 @@ bool launch_regs_are(const void* fn, int regs) {
 
 template <int D>
 fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, void* o, float* lse,
-                     int BH, int N, float scale, int causal, int o_f32, cudaStream_t stream) {
+                     int B, int H, int H_kv, int N, float scale, int causal, int o_f32, cudaStream_t stream) {
+  const int BH = B * H;
   using C = FwdCfg<D>;
   bool& attr = (D == 64) ? ds->fwd_attr64 : ds->fwd_attr128;
   if (!attr) {
@@ -137,7 +138,8 @@ fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, 
     attr = true;
   }
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, D, N, BH, 128) || !make_map(&tk, k, D, N, BH, 128) || !make_map(&tv, v, D, N, BH, 128))
+  if (!make_map(&tq, q, D, N, BH, 128) || !make_map(&tk, k, D, N, B * H_kv, 128) ||
+      !make_map(&tv, v, D, N, B * H_kv, 128))
     return FA_ERR_CUDA;
   FwdArgs a;
   a.o = o;
@@ -145,6 +147,8 @@ fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, 
   a.status = ds->status;
   a.N = N;
   a.bh = BH;
+  a.heads = H;
+  a.group = H / H_kv;
   a.n_qt = (N + 255) / 256;
   a.n_kv_all = (N + 127) / 128;
   a.num_tiles = BH * a.n_qt;
@@ -157,10 +161,12 @@ fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, 
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-                   float scale, int causal, fa_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream) {
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
+                   int d, float scale, int causal, fa_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream) {
   fa_status st = check_sizes(B, H, N, d, scale);
   if (st != FA_OK) return st;
+  if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID;
+  if (H_kv != H && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;   // grouped heads: bf16 inputs only
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
@@ -188,8 +194,8 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     vv = w + 2 * part;
   }
   const int of32 = dtype == FA_F32 ? 1 : 0;
-  return d == 64 ? launch_fwd<64>(ds, qq, kk, vv, o, lse, BH, N, scale, causal, of32, stream)
-                 : launch_fwd<128>(ds, qq, kk, vv, o, lse, BH, N, scale, causal, of32, stream);
+  return d == 64 ? launch_fwd<64>(ds, qq, kk, vv, o, lse, B, H, H_kv, N, scale, causal, of32, stream)
+                 : launch_fwd<128>(ds, qq, kk, vv, o, lse, B, H, H_kv, N, scale, causal, of32, stream);
 }
 
 }  // namespace
@@ -206,14 +212,20 @@ size_t fa_fwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype) {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  float scale, int causal, fa_stream_t stream) {
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, FA_BF16, nullptr, 0,
+  return fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, FA_BF16, nullptr, 0,
+                  static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                     int N, int d, float scale, int causal, fa_stream_t stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, FA_BF16, nullptr, 0,
                   static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                     float scale, int causal, fa_dtype dtype, void* workspace, size_t workspace_bytes,
                     fa_stream_t stream) {
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, workspace, workspace_bytes,
+  return fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, dtype, workspace, workspace_bytes,
                   static_cast<cudaStream_t>(stream));
 }
 
@@ -233,10 +245,11 @@ enum BwdPhase : int { PH_PREPARE = 1, PH_MAIN = 2, PH_FINISH = 4, PH_ALL = 7 };
 
 // Validates, fills the kernel arguments, and launches the requested phases.
 fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, const void* o, const float* lse,
-                   const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
-                   int causal, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                   const void* dout, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
+                   float scale, int causal, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   fa_status st = check_sizes(B, H, N, d, scale);
   if (st != FA_OK) return st;
+  if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID;
   if (d != 128) return FA_ERR_UNSUPPORTED;
   if ((phases & PH_PREPARE) && (!aligned16(o) || !aligned16(lse) || !aligned16(dout))) return FA_ERR_ALIGN;
   if ((phases & PH_MAIN) && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
@@ -273,11 +286,14 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   a.N = N;
   a.Np = static_cast<int>(np);
   a.bh = BH;
+  a.bh_kv = B * H_kv;
+  a.heads = H;
+  a.group = H / H_kv;
   a.n_kb = (N + 127) / 128;
   a.n_qb = (N + 127) / 128;
-  // enough heads per group to fill the GPU about twice over with key blocks
+  // enough key/value heads per scheduling group to fill the GPU about twice over with key blocks
   const int want = (2 * ds->sms + a.n_kb - 1) / a.n_kb;
-  a.heads_per_group = want < 1 ? 1 : (want > BH ? BH : want);
+  a.heads_per_group = want < 1 ? 1 : (want > a.bh_kv ? a.bh_kv : want);
   a.causal = causal ? 1 : 0;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
@@ -285,10 +301,10 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   if (phases & PH_PREPARE) fa_bwd_pre_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
   if (phases & PH_MAIN) {
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_map(&tq, q, d, N, BH, 128) || !make_map(&tk, k, d, N, BH, 128) ||
-        !make_map(&tv, v, d, N, BH, 128) || !make_map(&tdo, dout, d, N, BH, 128))
+    if (!make_map(&tq, q, d, N, BH, 128) || !make_map(&tk, k, d, N, a.bh_kv, 128) ||
+        !make_map(&tv, v, d, N, a.bh_kv, 128) || !make_map(&tdo, dout, d, N, BH, 128))
       return FA_ERR_CUDA;
-    fa_bwd_kernel<<<a.n_kb * BH, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    fa_bwd_kernel<<<a.n_kb * a.bh_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
   }
   if (phases & PH_FINISH) fa_bwd_dq_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -302,27 +318,34 @@ extern "C" {
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                  void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  return bwd_impl(PH_ALL, q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+  return bwd_impl(PH_ALL, q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, scale, causal, workspace,
+                  workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
+                     float scale, int causal, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  return bwd_impl(PH_ALL, q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, scale, causal, workspace,
                   workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_bwd_prepare(const void* o, const float* lse, const void* dout, int B, int H, int N, int d,
                          void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  return bwd_impl(PH_PREPARE, nullptr, nullptr, nullptr, o, lse, dout, nullptr, nullptr, nullptr, B, H, N, d,
+  return bwd_impl(PH_PREPARE, nullptr, nullptr, nullptr, o, lse, dout, nullptr, nullptr, nullptr, B, H, H, N, d,
                   1.0f, 0, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B,
                       int H, int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
                       fa_stream_t stream) {
-  return bwd_impl(PH_MAIN, q, k, v, nullptr, nullptr, dout, nullptr, dk, dv, B, H, N, d, scale, causal,
+  return bwd_impl(PH_MAIN, q, k, v, nullptr, nullptr, dout, nullptr, dk, dv, B, H, H, N, d, scale, causal,
                   workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_bwd_finish(void* dq, int B, int H, int N, int d, float scale, void* workspace,
                         size_t workspace_bytes, fa_stream_t stream) {
   return bwd_impl(PH_FINISH, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dq, nullptr, nullptr, B, H,
-                  N, d, scale, 0, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+                  H, N, d, scale, 0, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 // ---- backward with built-in scratch (no allocation) ----

@@ -38,7 +38,9 @@ struct FwdArgs {
   float* lse;           // [BH, N] natural-log logsumexp
   uint32_t* status;     // device status word
   int N;
-  int bh;               // B * H
+  int bh;               // B * H (query heads)
+  int heads;            // H
+  int group;            // query heads per key/value head (1: multi-head; H: multi-query)
   int n_qt;             // ceil(N / 256)
   int n_kv_all;         // ceil(N / 128)
   int num_tiles;        // bh * n_qt
@@ -85,6 +87,12 @@ __device__ __forceinline__ void fwd_decode_tile(const FwdArgs& a, int t, int& bh
     bh = t / a.n_qt;
     qt = t % a.n_qt;
   }
+}
+
+// Key/value head of query head bh: sets of `group` consecutive query heads of a
+// batch entry share one (grouped-query attention; group = 1 is multi-head).
+__device__ __forceinline__ int fwd_kv_head(const FwdArgs& a, int bh) {
+  return (bh / a.heads) * (a.heads / a.group) + (bh % a.heads) / a.group;
 }
 
 __device__ __forceinline__ int fwd_num_kv(const FwdArgs& a, int qt) {
@@ -159,6 +167,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         int bh, qt;
         fwd_decode_tile(args, t, bh, qt);
         const int nkv = fwd_num_kv(args, qt);
+        const int bh_kv = fwd_kv_head(args, bh);
         if (tile_cnt > 0 && !mbar_wait(b_q_empty, (tile_cnt - 1) & 1, ctl)) { ok = false; break; }
         mbar_expect_tx(b_q_full, 2 * C::Q_HALF);
         for (int h = 0; h < 2; ++h)
@@ -174,7 +183,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_expect_tx(b_kv_full(s), C::KV_BYTES);
             const CUtensorMap* map = kind ? &tm_v : &tm_k;
             for (int r = 0; r < C::N_REG; ++r)
-              tma_load_3d(sKV + s * C::KV_BYTES + r * C::REGION, map, b_kv_full(s), r * 64, j * 128, bh);
+              tma_load_3d(sKV + s * C::KV_BYTES + r * C::REGION, map, b_kv_full(s), r * 64, j * 128, bh_kv);
             issued |= 1u << s;
             last_parity = (last_parity & ~(1u << s)) | ((round & 1u) << s);
           }

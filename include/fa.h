@@ -118,6 +118,27 @@ fa_status fa_bwd_finish(void* dq, int B, int H, int N, int d, float scale,
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /*
+ * Grouped-query (and multi-query) attention: the nearauto.com FlashAttention-2
+ * digest, section "新機能: 最大256のヘッドディメンション、マルチクエリアテンション", has a
+ * set of query heads share one key/value head (the unite.ai page lists the
+ * same variants under "FlashAttention-2").  H query heads, H_kv key/value
+ * heads, H a multiple of H_kv; query head h of a batch entry reads key/value
+ * head h / (H / H_kv) (contiguous sets).  H_kv == H is fa_fwd / fa_bwd.
+ *  q, o, dO, dq: [B,H,N,d] bf16;  k, v, dk, dv: [B,H_kv,N,d] bf16;
+ *  lse: [B,H,N] float.  dk and dv of a shared head are the sums over its set.
+ * Same layout, ownership, alignment, stream and error rules as fa_fwd /
+ * fa_bwd, plus FA_ERR_INVALID when H_kv < 1 or H is not a multiple of H_kv.
+ * fa_bwd_gqa needs d == 128 and fa_bwd_workspace_size(B, H, N, d) bytes of
+ * workspace (sized by the query heads).
+ */
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int H_kv, int N, int d, float scale, int causal, fa_stream_t stream);
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv,
+                     int B, int H, int H_kv, int N, int d, float scale, int causal,
+                     void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * Backward without a caller-supplied workspace.  Same arguments, outputs and
  * numerics as fa_bwd, minus the workspace pair.  The paper has no counterpart
  * of this call; it exists for callers that cannot allocate device memory

@@ -73,6 +73,18 @@ def test_argument_validation_without_device(lib):
     assert b(*args, 1, 1, 128, 128, 0.125, 1, 16, need, None) == 4                 # not 256-aligned
 
 
+def test_grouped_query_validation_without_device(lib):
+    P16 = 16
+    f, b = lib.fa_fwd_gqa, lib.fa_bwd_gqa
+    assert f(P16, P16, P16, P16, P16, 1, 6, 4, 128, 64, 0.125, 0, None) == 1     # 6 heads over 4 sets
+    assert f(P16, P16, P16, P16, P16, 1, 6, 0, 128, 64, 0.125, 0, None) == 1     # no key/value head
+    assert f(P16, P16, P16, P16, P16 + 4, 1, 6, 2, 128, 64, 0.125, 0, None) == 3  # misaligned
+    args = [P16] * 9
+    assert b(*args, 1, 6, 4, 128, 128, 0.125, 1, P16, 1 << 30, None) == 1         # uneven sets
+    assert b(*args, 1, 6, 3, 128, 64, 0.125, 1, P16, 1 << 30, None) == 2          # d = 64
+    assert b(*args, 1, 6, 3, 128, 128, 0.125, 1, None, 0, None) == 4              # no workspace
+
+
 def test_workspace_sizes(lib):
     assert lib.fa_fwd_workspace_size(1, 1, 128, 64, 0) == 0
     assert lib.fa_fwd_workspace_size(1, 1, 128, 64, 1) == 3 * 128 * 64 * 2
