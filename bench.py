@@ -232,9 +232,13 @@ def is_fwd_only(args, w) -> bool:
 
 
 def workload_config(w, step: str, note: str):
-    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} {'causal' if w.causal else 'non-causal'}"
-                        + (f" K*{w.k_scale:g}" if w.k_scale != 1.0 else ""),
-            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "step": step, "l2": note}
+    c = {"workload": f"{w.name}: B={w.B} H={w.H}" + (f" H_kv={w.kv_heads}" if w.kv_heads != w.H else "")
+                     + f" N={w.N} d={w.d} {'causal' if w.causal else 'non-causal'}"
+                     + (f" K*{w.k_scale:g}" if w.k_scale != 1.0 else ""),
+         "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "step": step, "l2": note}
+    if w.kv_heads != w.H:
+        c["H_kv"] = w.kv_heads
+    return c
 
 
 # --------------------------------------------------------------------- GPU arm
@@ -270,7 +274,10 @@ def main():
     seed = w.seed + 100003 * rank          # each rank its own batch
     names = ("q", "k", "v") if fwd_only else ("q", "k", "v", "do")
     f32_in = w.dtype == "f32"               # fp32 inputs go through fa_fwd_ex (cast to bf16 on the GPU)
-    host = {n: inputs.make_tensor(seed, n, shape, w.k_scale if n == "k" else 1.0, "f32" if f32_in else "bf16")
+    gqa = w.kv_heads != w.H
+    kv_shape = (B, w.kv_heads, N, d)
+    host = {n: inputs.make_tensor(seed, n, kv_shape if n in ("k", "v") else shape, w.k_scale if n == "k" else 1.0,
+                                  "f32" if f32_in else "bf16")
             for n in names}
     if f32_in:
         pinned = {n: torch.from_numpy(host[n]).pin_memory() for n in names}
@@ -283,7 +290,8 @@ def main():
     if f32_in:
         fws = torch.empty(fa.fa_fwd_workspace_size(B, H, N, d, fa.FA_F32), dtype=torch.uint8, device=dev)
     if not fwd_only:
-        dq, dk, dvv = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
+        dq = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        dk, dvv = (torch.empty(kv_shape, dtype=torch.bfloat16, device=dev) for _ in range(2))
         ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     causal = w.causal
@@ -293,11 +301,21 @@ def main():
             ev[0].record(stream)
         if f32_in:
             fa.fa_fwd_ex(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, fa.FA_F32, fws, stream=stream)
+        elif gqa:
+            fa.fa_fwd_gqa(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, stream=stream)
         else:
             fa.fa_fwd(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, stream=stream)
         if ev is not None:
             ev[1].record(stream)
         if fwd_only:
+            return
+        if gqa:      # one call runs the three phases; its time is reported as the main kernel's
+            if ev is not None:
+                ev[2].record(stream)
+            fa.fa_bwd_gqa(dv_["q"], dv_["k"], dv_["v"], o, lse, dv_["do"], dq, dk, dvv, causal, ws, stream=stream)
+            if ev is not None:
+                ev[3].record(stream)
+                ev[4].record(stream)
             return
         fa.fa_bwd_prepare(o, lse, dv_["do"], ws, stream=stream)
         if ev is not None:
@@ -375,8 +393,11 @@ def main():
                                     "tflops": main_tf, "frac_of_measured_burst": main_tf / burst,
                                     "frac_of_measured_sustained": main_tf / sustained,
                                     "frac_of_datasheet": main_tf / DATASHEET_BF16_TFLOPS}
-        kernels["fa_bwd_pre_kernel"] = {"ms": prep_ms}
-        kernels["fa_bwd_dq_kernel"] = {"ms": fin_ms}
+        if gqa:
+            kernels["fa_bwd_kernel"]["note"] = "fa_bwd_gqa: prepare, main and finish kernels timed together"
+        else:
+            kernels["fa_bwd_pre_kernel"] = {"ms": prep_ms}
+            kernels["fa_bwd_dq_kernel"] = {"ms": fin_ms}
     dom = "fa_fwd_kernel" if (fwd_only or fwd_ms >= main_ms) else "fa_bwd_kernel"
     dom_flops = fwd_flops if dom == "fa_fwd_kernel" else bwd_flops
     achieved = kernels[dom]["tflops"]
@@ -386,7 +407,7 @@ def main():
                 "flops_per_launch": dom_flops, "traffic": committed_traffic(dom, w.name)}
     # forward HBM: each input read once, O and lse written once (the IO-aware minimum)
     in_elem = 4 if f32_in else 2
-    fwd_bytes = B * H * N * d * (3 * in_elem + o.element_size()) + 4 * B * H * N
+    fwd_bytes = B * N * d * (H * in_elem + 2 * w.kv_heads * in_elem + H * o.element_size()) + 4 * B * H * N
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     fwd_hbm = {"algorithmic_bytes": fwd_bytes, "gbs": fwd_bytes / (fwd_ms * 1e-3) / 1e9,
                "frac_of_measured_hbm": fwd_bytes / (fwd_ms * 1e-3) / 1e9 / hbm}

@@ -38,6 +38,11 @@ class Workload:
     k_scale: float      # K is multiplied by this before rounding
     seed: int
     backward: bool = False
+    h_kv: int = 0       # key/value heads (0: as many as query heads)
+
+    @property
+    def kv_heads(self) -> int:
+        return self.h_kv or self.H
 
     @property
     def scale(self) -> float:
@@ -55,6 +60,8 @@ WORKLOADS = {
     "prefill": Workload("prefill", 2, 32, 8192, 128, True, "bf16", 2.0, 1003),
     "long_context": Workload("long_context", 1, 16, 65536, 128, True, "bf16", 1.0, 1004),
     "backward": Workload("backward", 4, 16, 4096, 128, True, "bf16", 1.0, 1005, True),
+    # grouped-query attention on the prefill shape: 32 query heads over 8 key/value heads
+    "prefill_gqa": Workload("prefill_gqa", 2, 32, 8192, 128, True, "bf16", 2.0, 1006, False, 8),
 }
 
 
