@@ -6,6 +6,7 @@ from .attention import (  # noqa: F401
     attention_fwd,
     attention_fwd_gqa,
     attention_fwd_blockwise,
+    attention_fwd_decode,
     attention_fwd_rows,
     softmax_merge,
 )

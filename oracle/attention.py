@@ -41,6 +41,9 @@ Readings where the pages are silent or garbled (each is listed in the design doc):
     softmax(x u y) = [e^(m_x-m) l_x softmax(x), e^(m_y-m) l_y softmax(y)] / l;
   * the backward is the exact gradient of the forward (the pages only say
     "recompute"), with D_i = sum_j P_ij dP_ij;
+  * fewer queries than keys (decode, N_q < N_k): the queries are the last
+    N_q positions of the sequence, so causal query i sees keys j <= N_k - N_q + i
+    (bottom-right alignment; with N_q == N_k it is the usual mask);
   * grouped-query attention: the pages say each set of query heads shares one
     key/value head but not which; the sets are contiguous, query head h using
     key/value head h // (H / H_kv), and a shared head's gradient is the sum of
@@ -60,6 +63,7 @@ __all__ = [
     "attention_bwd",
     "attention_fwd_gqa",
     "attention_bwd_gqa",
+    "attention_fwd_decode",
     "softmax_merge",
     "attention_fwd_blockwise",
 ]
@@ -213,6 +217,35 @@ def attention_bwd_gqa(q, k, v, do, scale: float, causal: bool):
         dk[:, g] += dk_h[:, 0]
         dv[:, g] += dv_h[:, 0]
     return dq, dk, dv
+
+
+def attention_fwd_decode(q, k, v, scale: float, causal: bool):
+    """Attention of N_q queries against N_k >= N_q keys (decoding against a key/value cache).
+
+    q is [B, H, N_q, d]; k, v are [B, H_kv, N_k, d] (H a multiple of H_kv, as in
+    ``attention_fwd_gqa``).  The queries are the last N_q positions of the
+    sequence: causal query i sees keys j <= N_k - N_q + i.  Same definition as
+    ``attention_fwd`` otherwise ([P1] ``standard_attention``).  The decode
+    workload itself is the one the gist.science FlashAttention-V page times
+    ("decode"); splitting the keys and merging the partial results is [P1]'s
+    softmax merge.  Returns (O [B,H,N_q,d_v], lse [B,H,N_q]) in float64.
+    """
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    B, H, Nq, _ = q.shape
+    H_kv, Nk = k.shape[1], k.shape[2]
+    if Nq > Nk:
+        raise ValueError("more queries than keys")
+    rows = np.arange(Nk - Nq, Nk)
+    o = np.empty((B, H, Nq, v.shape[-1]), dtype=np.float64)
+    lse = np.empty((B, H, Nq), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            g = _kv_head(h, H, H_kv)
+            s = _scores(q[b, h], k[b, g], scale, rows, causal)
+            p, l_ = _softmax_rows(s)
+            o[b, h] = p @ v[b, g]
+            lse[b, h] = l_
+    return o, lse
 
 
 def softmax_merge(m_x, l_x, o_x, m_y, l_y, o_y):

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from oracle import (attention_bwd, attention_bwd_gqa, attention_fwd, attention_fwd_blockwise,
-                    attention_fwd_gqa, attention_fwd_rows, softmax_merge)
+                    attention_fwd_decode, attention_fwd_gqa, attention_fwd_rows, softmax_merge)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
@@ -324,6 +324,67 @@ def test_gqa_special_cases():
 def test_gqa_rejects_uneven_sets():
     with pytest.raises(ValueError):
         attention_fwd_gqa(_rand((1, 3, 4, 2), 1), _rand((1, 2, 4, 2), 2), _rand((1, 2, 4, 2), 3), 1.0, False)
+
+
+# --- decoding: fewer queries than keys, bottom-right causal alignment ------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_decode_matches_torch_sdpa_with_explicit_mask(causal):
+    """torch SDPA (float64) with an explicit bottom-right boolean mask and enable_gqa."""
+    B, H, H_kv, Nq, Nk, d, scale = 2, 4, 2, 5, 37, 8, 0.35
+    q = _rand((B, H, Nq, d), 121)
+    k, v = _rand((B, H_kv, Nk, d), 122), _rand((B, H_kv, Nk, d), 123)
+    o, lse = attention_fwd_decode(q, k, v, scale, causal)
+    mask = None
+    if causal:
+        mask = torch.ones(Nq, Nk, dtype=torch.bool).tril(Nk - Nq)     # query i sees j <= Nk - Nq + i
+    to = torch.nn.functional.scaled_dot_product_attention(torch.tensor(q), torch.tensor(k), torch.tensor(v),
+                                                          attn_mask=mask, scale=scale, enable_gqa=True)
+    np.testing.assert_allclose(o, to.numpy(), atol=1e-12)
+    s = scale * torch.tensor(q) @ torch.tensor(k).repeat_interleave(H // H_kv, 1).transpose(-1, -2)
+    if causal:
+        s = s.masked_fill(~mask, float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), atol=1e-12)
+
+
+def test_decode_special_cases():
+    """N_q == N_k is the square (top-left == bottom-right) case; one query, or the last
+    query of any causal decode, sees every key."""
+    q, k, v = (_rand((1, 4, 23, 8), 130 + i) for i in range(3))
+    for causal in (False, True):
+        o, lse = attention_fwd_decode(q, k[:, :2], v[:, :2], 0.3, causal)
+        o1, lse1 = attention_fwd_gqa(q, k[:, :2], v[:, :2], 0.3, causal)
+        np.testing.assert_allclose(o, o1, atol=1e-14)
+        np.testing.assert_allclose(lse, lse1, atol=1e-14)
+    q4 = _rand((1, 4, 6, 8), 140)
+    oc, lc = attention_fwd_decode(q4, k, v, 0.3, True)
+    on, ln = attention_fwd_decode(q4, k, v, 0.3, False)
+    np.testing.assert_allclose(oc[:, :, -1], on[:, :, -1], atol=1e-14)
+    np.testing.assert_allclose(lc[:, :, -1], ln[:, :, -1], atol=1e-14)
+    assert not np.allclose(oc[:, :, 0], on[:, :, 0])
+    o1c, _ = attention_fwd_decode(q4[:, :, :1], k, v, 0.3, True)
+    o1n, _ = attention_fwd_decode(q4[:, :, :1], k, v, 0.3, False)
+    np.testing.assert_allclose(o1c, o1n, atol=1e-14)
+
+
+def test_decode_split_keys_merge_to_the_whole():
+    """Partial results over disjoint key ranges, merged with softmax_merge, give the
+    whole decode result (the split-KV structure, in the oracle's own terms)."""
+    q = _rand((1, 2, 3, 8), 150)
+    k, v = _rand((1, 1, 50, 8), 151, 2.0), _rand((1, 1, 50, 8), 152)
+    o, lse = attention_fwd_decode(q, k, v, 0.4, False)
+    parts = [(0, 17), (17, 40), (40, 50)]
+    m_acc, l_acc, o_acc = None, None, None
+    for a, b in parts:
+        op, lp = attention_fwd_decode(q, k[:, :, a:b], v[:, :, a:b], 0.4, False)
+        m_p, l_p = lp.reshape(-1), np.ones(lp.size)          # lse as the max with l = 1
+        o_p = op.reshape(-1, 8)
+        if m_acc is None:
+            m_acc, l_acc, o_acc = m_p, l_p, o_p
+        else:
+            m_acc, l_acc, o_acc = softmax_merge(m_acc, l_acc, o_acc, m_p, l_p, o_p)
+    np.testing.assert_allclose(o_acc, o.reshape(-1, 8), atol=1e-13)
+    np.testing.assert_allclose(m_acc + np.log(l_acc), lse.reshape(-1), atol=1e-13)
 
 
 # --- the softmax merge and the blockwise algorithm -------------------------
