@@ -24,6 +24,7 @@ FA_BF16, FA_F32 = 0, 1
 EXPORTS = (
     "fa_fwd", "fa_fwd_ex", "fa_fwd_workspace_size", "fa_bwd", "fa_bwd_workspace_size",
     "fa_bwd_prepare", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc", "fa_fwd_gqa", "fa_bwd_gqa",
+    "fa_decode", "fa_decode_workspace_size",
     "fa_get_device_status", "fa_selftest_wait_timeout", "fa_status_string", "fa_version",
 )
 
@@ -57,6 +58,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P]
     L.fa_fwd_gqa.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P]
     L.fa_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, Z, P]
+    L.fa_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, Z, P]
+    L.fa_decode_workspace_size.argtypes = [I, I, I, I, I, I]
+    L.fa_decode_workspace_size.restype = Z
     L.fa_bwd_workspace_size.argtypes = [I, I, I, I]
     L.fa_bwd_workspace_size.restype = Z
     L.fa_get_device_status.argtypes = [P]
@@ -65,7 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_version.restype = ctypes.c_char_p
     for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_prepare", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc",
-                 "fa_fwd_gqa", "fa_bwd_gqa", "fa_get_device_status", "fa_selftest_wait_timeout"):
+                 "fa_fwd_gqa", "fa_bwd_gqa", "fa_decode", "fa_get_device_status", "fa_selftest_wait_timeout"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -196,6 +200,33 @@ def fa_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, workspace, scale
     _check(load_library().fa_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
                                      _ptr(dk), _ptr(dv), B, H, H_kv, N, d, scale, int(bool(causal)),
                                      _ptr(workspace), _ws_bytes(workspace), _stream(stream)), "fa_bwd_gqa")
+
+
+def fa_decode_workspace_size(B: int, H: int, H_kv: int, Lq: int, Nk: int, d: int) -> int:
+    return int(load_library().fa_decode_workspace_size(B, H, H_kv, Lq, Nk, d))
+
+
+def fa_decode(q, k, v, o, lse, causal: bool, workspace, scale: float | None = None, stream=None) -> None:
+    """Decode: q, o [B,H,Lq,d] (the last Lq positions); k, v [B,H_kv,Nk,d]; lse [B,H,Lq]."""
+    B, H, Lq, d = _bhnd(q)
+    _, H_kv, Nk, _ = _bhnd(k)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(load_library().fa_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, H_kv, Lq, Nk, d, scale,
+                                    int(bool(causal)), _ptr(workspace), _ws_bytes(workspace), _stream(stream)),
+           "fa_decode")
+
+
+def decode(q, k, v, causal: bool, scale: float | None = None, stream=None, workspace=None):
+    """O, lse of the last Lq query positions q [B,H,Lq,d] against a cache k, v [B,H_kv,Nk,d] (bf16)."""
+    import torch
+    B, H, Lq, d = _bhnd(q)
+    _, H_kv, Nk, _ = _bhnd(k)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(fa_decode_workspace_size(B, H, H_kv, Lq, Nk, d), q.device)
+    fa_decode(q, k, v, o, lse, causal, workspace, scale, stream)
+    return o, lse
 
 
 def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:

@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "bwd_kernel.cuh"
+#include "decode_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace fa {
@@ -25,7 +26,7 @@ struct DevState {
   bool ready = false;
   uint32_t* status = nullptr;
   int sms = 0;
-  bool fwd_attr64 = false, fwd_attr128 = false, bwd_attr = false;
+  bool fwd_attr64 = false, fwd_attr128 = false, bwd_attr = false, dec_attr = false;
 };
 DevState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -402,6 +403,66 @@ fa_status fa_selftest_wait_timeout(uint64_t timeout_ns, fa_stream_t stream) {
   uint64_t t = timeout_ns < 1000000ull ? 1000000ull : timeout_ns;
   if (t > kWaitLimitNs) t = kWaitLimitNs;
   wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ds->status, t);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_decode_workspace_size(int B, int H, int H_kv, int Lq, int Nk, int d) {
+  if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || Lq < 1 || Nk < Lq || d < 1) return 0;
+  int split_keys = 0;
+  const size_t splits = static_cast<size_t>(decode_splits(B * H_kv, Nk, &split_keys));
+  const size_t rows = static_cast<size_t>(B) * H * Lq;
+  return round256(splits * rows * d * 4) + round256(splits * rows * 4);
+}
+
+fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                    int Lq, int Nk, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                    fa_stream_t stream) {
+  fa_status st = check_sizes(B, H_kv, Nk, d, scale);
+  if (st != FA_OK) return st;
+  if (Lq < 1 || Lq > Nk || H < 1 || H_kv > H || H % H_kv != 0 || 1LL * B * H * Lq * d >= (1LL << 31) ||
+      B * H_kv > 65535)
+    return FA_ERR_INVALID;
+  if (d != DecCfg::D || (H / H_kv) * Lq > DecCfg::R_MAX) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
+  const size_t need = fa_decode_workspace_size(B, H, H_kv, Lq, Nk, d);
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return FA_ERR_WORKSPACE;
+  DevState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  if (!ds->dec_attr) {
+    if (cudaFuncSetAttribute(fa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg::SMEM_BYTES) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    ds->dec_attr = true;
+  }
+  CUtensorMap tk, tv;
+  if (!make_map(&tk, k, d, Nk, B * H_kv, DecCfg::KT) || !make_map(&tv, v, d, Nk, B * H_kv, DecCfg::KT))
+    return FA_ERR_CUDA;
+  DecArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = ds->status;
+  a.Lq = Lq;
+  a.Nk = Nk;
+  a.heads = H;
+  a.group = H / H_kv;
+  a.bh = B * H;
+  a.bh_kv = B * H_kv;
+  a.n_splits = decode_splits(a.bh_kv, Nk, &a.split_keys);
+  a.causal = causal ? 1 : 0;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.wait_limit_ns = kWaitLimitNs;
+  const size_t rows = static_cast<size_t>(a.bh) * Lq;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  a.part_o = reinterpret_cast<float*>(w);
+  a.part_lse = reinterpret_cast<float*>(w + round256(static_cast<size_t>(a.n_splits) * rows * d * 4));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fa_decode_kernel<<<dim3(a.n_splits, a.bh_kv), DecCfg::THREADS, DecCfg::SMEM_BYTES, s>>>(tk, tv, a);
+  const size_t warps = rows, per_block = 8;
+  size_t blocks = (warps + per_block - 1) / per_block;
+  if (blocks > static_cast<size_t>(ds->sms) * 16) blocks = static_cast<size_t>(ds->sms) * 16;
+  fa_decode_merge_kernel<<<static_cast<unsigned>(blocks), 32 * per_block, 0, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -139,6 +139,29 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
                      void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Decoding: Lq queries that are the last Lq positions of a sequence of Nk keys
+ * (a key/value cache), with the keys split across CTAs and the partial results
+ * combined by the softmax merge of the unite.ai page "Flash Attention:
+ * Rivoluzionando l'Efficienza dei Modelli Transformer", section "La Matematica
+ * dietro Flash Attention".  The decode workload is the one the gist.science
+ * FlashAttention-V page times.
+ *  q, o: [B,H,Lq,d] bf16;  k, v: [B,H_kv,Nk,d] bf16 (H a multiple of H_kv, as
+ *  in fa_fwd_gqa);  lse: [B,H,Lq] float (natural log).
+ *  causal != 0: query i sees keys j <= Nk - Lq + i (bottom-right alignment).
+ * Needs d == 128 and (H / H_kv) * Lq <= 16 (FA_ERR_UNSUPPORTED otherwise),
+ * 1 <= Lq <= Nk and B * H_kv <= 65535 (FA_ERR_INVALID).  workspace: at least
+ * fa_decode_workspace_size(...) bytes, 256-byte aligned (the per-split partial
+ * outputs); same layout, ownership, alignment, stream and error rules as
+ * fa_fwd otherwise.  Two kernels: the split partials, then the merge.
+ */
+fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int H, int H_kv, int Lq, int Nk, int d, float scale, int causal,
+                    void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/* Bytes of workspace fa_decode needs (0 for invalid sizes). */
+size_t fa_decode_workspace_size(int B, int H, int H_kv, int Lq, int Nk, int d);
+
+/*
  * Backward without a caller-supplied workspace.  Same arguments, outputs and
  * numerics as fa_bwd, minus the workspace pair.  The paper has no counterpart
  * of this call; it exists for callers that cannot allocate device memory

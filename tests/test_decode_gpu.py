@@ -1,0 +1,68 @@
+"""Decode (few queries against a key/value cache, split keys merged) on the GPU
+against the fp64 oracle's attention_fwd_decode.  Same tolerances as the forward."""
+import numpy as np
+import pytest
+
+from exact_io_aware_100_b200 import inputs
+from helpers import assert_close, assert_lse, to_device, to_f64
+from oracle import attention_fwd_decode
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(B, H, H_kv, Lq, Nk, seed, k_scale=1.0):
+    d = 128
+    host = {"q": inputs.make_tensor(seed, "q", (B, H, Lq, d)),
+            "k": inputs.make_tensor(seed, "k", (B, H_kv, Nk, d), k_scale),
+            "v": inputs.make_tensor(seed, "v", (B, H_kv, Nk, d))}
+    f64 = {n: inputs.to_f64(x, "bf16") for n, x in host.items()}
+    return host, f64
+
+
+@pytest.mark.parametrize("B,H,H_kv,Lq,Nk,causal", [
+    (2, 8, 2, 1, 1000, True),       # one token, grouped heads
+    (1, 4, 4, 1, 4096, False),      # plain multi-head
+    (2, 8, 1, 2, 777, True),        # multi-query, two tokens, ragged cache
+    (1, 4, 1, 4, 63, True),         # cache shorter than one tile
+    (1, 2, 2, 16, 2049, True),      # 16 tokens per head (causal bottom-right inside the last tile)
+    (3, 6, 3, 8, 5000, False),
+    (1, 16, 2, 2, 65536, True),     # long cache: many splits
+])
+def test_decode_matches_oracle(B, H, H_kv, Lq, Nk, causal):
+    import torch
+    import exact_io_aware_100_b200 as fa
+    host, f64 = _case(B, H, H_kv, Lq, Nk, 3100 + Lq + Nk % 97)
+    q, k, v = (to_device(host[n], "bf16") for n in ("q", "k", "v"))
+    o, lse = fa.decode(q, k, v, causal)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == fa.FA_OK
+    ro, rl = attention_fwd_decode(f64["q"], f64["k"], f64["v"], 1.0 / np.sqrt(128), causal)
+    assert_close("O", to_f64(o), ro)
+    assert_lse(to_f64(lse), rl)
+
+
+def test_decode_sharp_scores():
+    """K scaled by 4: sharp softmax rows, the split partials differ by many e-folds."""
+    import torch
+    import exact_io_aware_100_b200 as fa
+    host, f64 = _case(1, 8, 2, 1, 3000, 3200, k_scale=4.0)
+    q, k, v = (to_device(host[n], "bf16") for n in ("q", "k", "v"))
+    o, lse = fa.decode(q, k, v, True)
+    torch.cuda.synchronize()
+    ro, rl = attention_fwd_decode(f64["q"], f64["k"], f64["v"], 1.0 / np.sqrt(128), True)
+    assert_close("O", to_f64(o), ro)
+    assert_lse(to_f64(lse), rl, tol=1e-3 * 16)
+
+
+def test_decode_of_the_whole_sequence_matches_the_forward():
+    """Lq == Nk is ordinary causal attention: decode equals the forward kernel's result
+    within the forward tolerance."""
+    import torch
+    import exact_io_aware_100_b200 as fa
+    host, _ = _case(1, 4, 4, 16, 16, 3300)
+    q, k, v = (to_device(host[n], "bf16") for n in ("q", "k", "v"))
+    o1, l1 = fa.decode(q, k, v, True)
+    o2, l2 = fa.forward(q, k, v, True)
+    torch.cuda.synchronize()
+    assert_close("O", to_f64(o1), to_f64(o2))
+    assert_lse(to_f64(l1), to_f64(l2).astype(np.float64))
