@@ -172,9 +172,20 @@ class ClockSampler:
 def oracle_sample(w, heads: int, seed_offset: int = 0, fwd_only: bool = False):
     """fwd (+ bwd) of `heads` whole heads of the workload with the fp64 oracle.
     Returns (seconds, algorithmic FLOPs of the sample, description)."""
-    from oracle import attention_bwd, attention_fwd
+    from oracle import attention_bwd, attention_fwd, attention_fwd_decode
     shape1 = (1, 1, w.N, w.d)
     t_total, flops = 0.0, 0.0
+    if w.lq:       # decode: one query head's lq positions against its cache
+        for i in range(heads):
+            seed = w.seed + 7919 * (i + 1 + seed_offset)
+            f = {n: inputs.to_f64(inputs.make_tensor(seed, n, (1, 1, w.lq if n == "q" else w.N, w.d)), "bf16")
+                 for n in ("q", "k", "v")}
+            t0 = time.perf_counter()
+            attention_fwd_decode(f["q"], f["k"], f["v"], w.scale, w.causal)
+            t_total += time.perf_counter() - t0
+            flops += w.fwd_flops() / (w.B * w.H)
+        return t_total, flops, (f"decode of {heads} query head(s) ({w.lq} x {w.d} against {w.N} keys), "
+                                f"numpy float64 oracle")
     for i in range(heads):
         seed = w.seed + 7919 * (i + 1 + seed_offset)
         f = {n: inputs.to_f64(inputs.make_tensor(seed, n, shape1, w.k_scale if n == "k" else 1.0), "bf16")
@@ -228,20 +239,129 @@ def run_reference(args, w):
 
 def is_fwd_only(args, w) -> bool:
     """The backward kernel covers d = 128 with bf16 inputs; other workloads time the forward."""
-    return args.fwd_only or w.d != 128 or w.dtype != "bf16"
+    return args.fwd_only or w.d != 128 or w.dtype != "bf16" or bool(w.lq)
 
 
 def workload_config(w, step: str, note: str):
     c = {"workload": f"{w.name}: B={w.B} H={w.H}" + (f" H_kv={w.kv_heads}" if w.kv_heads != w.H else "")
+                     + (f" Lq={w.lq}" if w.lq else "")
                      + f" N={w.N} d={w.d} {'causal' if w.causal else 'non-causal'}"
                      + (f" K*{w.k_scale:g}" if w.k_scale != 1.0 else ""),
          "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "step": step, "l2": note}
     if w.kv_heads != w.H:
         c["H_kv"] = w.kv_heads
+    if w.lq:
+        c["Lq"] = w.lq
     return c
 
 
 # --------------------------------------------------------------------- GPU arm
+def run_decode(args, w, fa, torch, dist, world, rank, local_rank, dev):
+    """Decode workloads: fa_decode (split partials + merge) over a cache larger than L2; HBM bound."""
+    B, H, Hkv, Lq, N, d = w.B, w.H, w.kv_heads, w.lq, w.N, w.d
+    seed = w.seed + 100003 * rank
+    shapes = {"q": (B, H, Lq, d), "k": (B, Hkv, N, d), "v": (B, Hkv, N, d)}
+    host = {n: inputs.make_tensor(seed, n, shp) for n, shp in shapes.items()}
+    pinned = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in host}
+    dv_ = {n: pinned[n].to(dev) for n in host}
+    o = torch.empty(shapes["q"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, Lq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_decode_workspace_size(B, H, Hkv, Lq, N, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    io_bytes = sum(x.nbytes for x in host.values()) + o.numel() * 2 + lse.numel() * 4
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if io_bytes < 2 * L2_BYTES else None
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fa.fa_decode(dv_["q"], dv_["k"], dv_["v"], o, lse, w.causal, ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_get_device_status() != fa.FA_OK:
+        raise SystemExit("device status reported a timeout during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            if flush is not None:
+                flush.fill_(s & 0xff)
+            step(evs[s])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    elapsed_ms = sum(step_ms) if flush is not None else t0.elapsed_time(t1)
+    if fa.fa_get_device_status() != fa.FA_OK:
+        raise SystemExit("device status reported a timeout in the timed region")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    flops = w.fwd_flops()
+    value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    dec_ms = statistics.mean(step_ms)
+    gbs = io_bytes / (dec_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "fa_decode_kernel + fa_decode_merge_kernel", "achieved": gbs,
+                "peak": hbm, "unit": "GB/s", "frac": gbs / hbm, "peak_source": f"{peak_src} hbm_gbs",
+                "bytes_per_launch": io_bytes, "traffic": None}
+    e2e = None
+    if not args.no_e2e:
+        host_out = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
+                    "lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)}
+
+        def e2e_step():
+            for n in host:
+                dv_[n].copy_(pinned[n], non_blocking=True)
+            step()
+            host_out["o"].copy_(o, non_blocking=True)
+            host_out["lse"].copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        e2e = {"value": world * flops * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(x.nbytes for x in host.values()),
+               "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4, "ms_per_step": e_ms / args.e2e_steps}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, f, desc = oracle_sample(w, args.cpu_heads)
+        cpu = {"value": f / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc + f"; {secs:.1f} s"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, "decode",
+                                  f"cache larger than L2 ({io_bytes / 2**20:.0f} MiB per step), no flush"
+                                  if flush is None else "L2 flushed before every step"),
+        "kernels": {"fa_decode": {"ms": dec_ms, "median_ms": statistics.median(step_ms), "min_ms": min(step_ms),
+                                  "gbs": gbs, "frac_of_measured_hbm": gbs / hbm}},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": 2 * args.steps, "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     w = inputs.WORKLOADS[args.workload]
@@ -267,6 +387,9 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     fa.load_library()
+    if w.lq:
+        run_decode(args, w, fa, torch, dist, world, rank, local_rank, dev)
+        return
 
     fwd_only = is_fwd_only(args, w)
     B, H, N, d = w.B, w.H, w.N, w.d

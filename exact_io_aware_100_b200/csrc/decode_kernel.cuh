@@ -20,9 +20,12 @@
 //    rows are the N_q queries of every query head of the key/value head's set
 //    (at most 16 rows).  64-key tiles of K and V stream through a two-stage
 //    TMA ring (128-byte swizzle, so per-lane shared reads are conflict free).
-//    Warp w owns rows w and w + 8; for scores each lane takes two keys, for
-//    P.V each lane four of the 128 output columns.  Writes the split's
-//    normalised partial O (fp32) and its lse (-inf when no key is visible);
+//    Per tile, every warp works whatever the row count: scores with one thread
+//    per (key, group of rows), the online softmax with one warp per row, and
+//    P.V with each warp taking 8 of the 64 keys for all rows (four output
+//    columns per lane), keeping a partial O over its keys that the warps sum
+//    once at the end of the split.  Writes the split's normalised partial O
+//    (fp32) and its lse (-inf when no key is visible);
 //  * fa_decode_merge_kernel:  one warp per query row, merges the splits.
 #pragma once
 
@@ -54,10 +57,12 @@ struct DecCfg {
   static constexpr int THREADS = 256;
   static constexpr int KREG = KT * 128;          // one 64-column swizzle region of a 64-row tile
   static constexpr int TILE = 2 * KREG;          // a 64 x 128 bf16 tile (16 KB)
-  static constexpr int OFF_Q = 0;                // fp32 [R_MAX][D]
+  static constexpr int OFF_Q = 0;                // fp32 [R_MAX][D]; reused to sum the warps' partial O
   static constexpr int OFF_ST = R_MAX * D * 4;   // two stages of K then V
   static constexpr int STAGE = 2 * TILE;
-  static constexpr int OFF_BAR = OFF_ST + 2 * STAGE;
+  static constexpr int OFF_S = OFF_ST + 2 * STAGE;          // fp32 [R_MAX][KT]: scores, then P
+  static constexpr int OFF_ROW = OFF_S + R_MAX * KT * 4;    // fp32 [R_MAX]: alpha of the tile, then l
+  static constexpr int OFF_BAR = OFF_ROW + R_MAX * 4;
   static constexpr int OFF_MISC = OFF_BAR + 16;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
 };
@@ -74,7 +79,9 @@ __host__ __device__ inline int decode_splits(int bh_kv, int Nk, int* split_keys)
   return (tiles + tiles_per - 1) / tiles_per;
 }
 
-__global__ void __launch_bounds__(DecCfg::THREADS)
+// RM: a bound on the rows (4, 8 or 16), which sizes the partial-O registers.
+template <int RM>
+__global__ void __launch_bounds__(DecCfg::THREADS, 2)
 fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const DecArgs a) {
   using C = DecCfg;
@@ -128,14 +135,21 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (n_tiles > 1) issue(1);
   }
 
-  // this warp's rows and their causal limits (key positions <= lim are visible)
-  const int ra = warp, rb = warp + 8;
-  const bool va = ra < R, vb = rb < R;
-  const int lim_a = a.causal ? a.Nk - a.Lq + ra % a.Lq : a.Nk - 1;
-  const int lim_b = a.causal ? a.Nk - a.Lq + rb % a.Lq : a.Nk - 1;
+  float* ss = reinterpret_cast<float*>(smem + C::OFF_S);     // [R_MAX][KT]
+  float* srow = reinterpret_cast<float*>(smem + C::OFF_ROW); // [R_MAX]
   const float c2 = a.scale_log2;
+  // causal limit of row r: key positions <= lim are visible
+  auto lim_of = [&](int r) { return a.causal ? a.Nk - a.Lq + r % a.Lq : a.Nk - 1; };
+  // scores: thread = (key sk, rows sr0, sr0 + 4, sr0 + 8, sr0 + 12)
+  const int sk = tid & (C::KT - 1), sr0 = tid >> 6;
+  // softmax: warp w owns rows w and w + 8 (running max m and sum l)
+  const int ra = warp, rb = warp + 8;
   float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-  float oa[4] = {0.f, 0.f, 0.f, 0.f}, ob[4] = {0.f, 0.f, 0.f, 0.f};
+  // P.V: warp w takes keys 8w .. 8w + 7 of every tile; lane owns columns 4 lane .. 4 lane + 3
+  float acc[RM][4];
+#pragma unroll
+  for (int r = 0; r < RM; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+  const int pj = lane >> 1, pregion = pj >> 3, pc = pj & 7;
   bool ok = true;
   int t_fail = n_tiles;
   for (int t = 0; t < n_tiles; ++t) {
@@ -143,92 +157,95 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (!__syncthreads_and(ok)) { ok = false; t_fail = t; break; }   // every thread agrees before using the stage
     const uint8_t* st = smem + C::OFF_ST + (t & 1) * C::STAGE;
     const int kt0 = k_begin + t * C::KT;
-    if (va) {
-      // scores of rows ra, rb against keys lane and lane + 32
-      float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
-      const int k0 = lane, k1 = lane + 32;
+    // ---- scores S[r][sk] for this thread's rows (row groups beyond R do nothing)
+    if (sr0 < R) {
+      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 16; ++j) {        // 16-byte chunks along d
-        const int region = j >> 3, c = j & 7;
-        const uint4 w0 = *reinterpret_cast<const uint4*>(st + region * C::KREG + k0 * 128 + ((c ^ (k0 & 7)) << 4));
-        const uint4 w1 = *reinterpret_cast<const uint4*>(st + region * C::KREG + k1 * 128 + ((c ^ (k1 & 7)) << 4));
-        const uint32_t ka[4] = {w0.x, w0.y, w0.z, w0.w}, kb[4] = {w1.x, w1.y, w1.z, w1.w};
-        const float4 qa0 = *reinterpret_cast<const float4*>(sq + ra * D + 8 * j);
-        const float4 qa1 = *reinterpret_cast<const float4*>(sq + ra * D + 8 * j + 4);
-        const float4 qb0 = *reinterpret_cast<const float4*>(sq + (vb ? rb : ra) * D + 8 * j);
-        const float4 qb1 = *reinterpret_cast<const float4*>(sq + (vb ? rb : ra) * D + 8 * j + 4);
-        const float qa[8] = {qa0.x, qa0.y, qa0.z, qa0.w, qa1.x, qa1.y, qa1.z, qa1.w};
-        const float qb[8] = {qb0.x, qb0.y, qb0.z, qb0.w, qb1.x, qb1.y, qb1.z, qb1.w};
+        const uint4 w = *reinterpret_cast<const uint4*>(st + (j >> 3) * C::KREG + sk * 128 + (((j & 7) ^ (sk & 7)) << 4));
+        float kf[8];
+        const uint32_t kw[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ka[e]));
-          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kb[e]));
-          sa0 = fmaf(qa[2 * e], f0.x, fmaf(qa[2 * e + 1], f0.y, sa0));
-          sa1 = fmaf(qa[2 * e], f1.x, fmaf(qa[2 * e + 1], f1.y, sa1));
-          if (vb) {                          // warp-uniform: a second row only when the set has one
-            sb0 = fmaf(qb[2 * e], f0.x, fmaf(qb[2 * e + 1], f0.y, sb0));
-            sb1 = fmaf(qb[2 * e], f1.x, fmaf(qb[2 * e + 1], f1.y, sb1));
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw[e]));
+          kf[2 * e] = f.x;
+          kf[2 * e + 1] = f.y;
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int r = sr0 + 4 * g;
+          if (r < R) {                        // uniform across the warp
+            const float4 q0 = *reinterpret_cast<const float4*>(sq + r * D + 8 * j);
+            const float4 q1 = *reinterpret_cast<const float4*>(sq + r * D + 8 * j + 4);
+            float x = sacc[g];
+            x = fmaf(q0.x, kf[0], x); x = fmaf(q0.y, kf[1], x); x = fmaf(q0.z, kf[2], x); x = fmaf(q0.w, kf[3], x);
+            x = fmaf(q1.x, kf[4], x); x = fmaf(q1.y, kf[5], x); x = fmaf(q1.z, kf[6], x); x = fmaf(q1.w, kf[7], x);
+            sacc[g] = x;
           }
         }
       }
-      // mask: keys past the split (or the cache) and, causal, after the query's position
-      const int p0 = kt0 + k0, p1 = kt0 + k1;
-      if (p0 >= k_end || p0 > lim_a) sa0 = -INFINITY;
-      if (p1 >= k_end || p1 > lim_a) sa1 = -INFINITY;
-      if (!vb || p0 >= k_end || p0 > lim_b) sb0 = -INFINITY;
-      if (!vb || p1 >= k_end || p1 > lim_b) sb1 = -INFINITY;
-      // online softmax, per row, over the warp's 64 keys
-      float ta = fmaxf(sa0, sa1), tb = fmaxf(sb0, sb1);
+      const int pos = kt0 + sk;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, off));
-        tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, off));
+      for (int g = 0; g < 4; ++g) {
+        const int r = sr0 + 4 * g;
+        if (r < R) ss[r * C::KT + sk] = (pos < k_end && pos <= lim_of(r)) ? sacc[g] : -INFINITY;
       }
-      const float mna = fmaxf(m_a, ta), mnb = fmaxf(m_b, tb);
-      // rows that have seen no visible key keep m = -inf and contribute nothing
-      const float alpha_a = (mna == -INFINITY) ? 1.f : ex2_approx((m_a - mna) * c2);
-      const float alpha_b = (mnb == -INFINITY) ? 1.f : ex2_approx((m_b - mnb) * c2);
-      const float na = (mna == -INFINITY) ? 0.f : mna * c2, nb = (mnb == -INFINITY) ? 0.f : mnb * c2;
-      const float pa0 = ex2_approx(fmaf(sa0, c2, -na)), pa1 = ex2_approx(fmaf(sa1, c2, -na));
-      const float pb0 = ex2_approx(fmaf(sb0, c2, -nb)), pb1 = ex2_approx(fmaf(sb1, c2, -nb));
-      float suma = pa0 + pa1, sumb = pb0 + pb1;
+    }
+    __syncthreads();
+    // ---- online softmax: rows ra and rb of this warp; P back into ss, the tile's alpha into srow
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        suma += __shfl_xor_sync(0xffffffffu, suma, off);
-        sumb += __shfl_xor_sync(0xffffffffu, sumb, off);
-      }
-      l_a = l_a * alpha_a + suma;
-      l_b = l_b * alpha_b + sumb;
-      m_a = mna;
-      m_b = mnb;
+    for (int h = 0; h < 2; ++h) {
+      const int r = h ? rb : ra;
+      if (r < R) {
+        float& m = h ? m_b : m_a;
+        float& l = h ? l_b : l_a;
+        const float s0 = ss[r * C::KT + lane], s1 = ss[r * C::KT + lane + 32];
+        float mt = fmaxf(s0, s1);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        oa[e] *= alpha_a;
-        ob[e] *= alpha_b;
+        for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+        const float mn = fmaxf(m, mt);
+        // a row that has seen no visible key keeps m = -inf and contributes nothing
+        const float alpha = (mn == -INFINITY) ? 1.f : ex2_approx((m - mn) * c2);
+        const float nb = (mn == -INFINITY) ? 0.f : mn * c2;
+        const float p0 = ex2_approx(fmaf(s0, c2, -nb)), p1 = ex2_approx(fmaf(s1, c2, -nb));
+        float sum = p0 + p1;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        l = l * alpha + sum;
+        m = mn;
+        ss[r * C::KT + lane] = p0;
+        ss[r * C::KT + lane + 32] = p1;
+        if (lane == 0) srow[r] = alpha;
       }
-      // O += P V: lane owns output columns 4 lane .. 4 lane + 3 (16-byte chunk lane / 2, half lane % 2)
-      const int j = lane >> 1, region = j >> 3, c = j & 7;
-      const uint8_t* vbase = st + C::TILE + region * C::KREG + (lane & 1) * 8;
-#pragma unroll 8
-      for (int k = 0; k < C::KT; ++k) {
-        const float pk_a = __shfl_sync(0xffffffffu, k < 32 ? pa0 : pa1, k & 31);
-        const uint2 w = *reinterpret_cast<const uint2*>(vbase + k * 128 + ((c ^ (k & 7)) << 4));
-        const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
-        const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
-        oa[0] = fmaf(pk_a, v01.x, oa[0]);
-        oa[1] = fmaf(pk_a, v01.y, oa[1]);
-        oa[2] = fmaf(pk_a, v23.x, oa[2]);
-        oa[3] = fmaf(pk_a, v23.y, oa[3]);
-        if (vb) {
-          const float pk_b = __shfl_sync(0xffffffffu, k < 32 ? pb0 : pb1, k & 31);
-          ob[0] = fmaf(pk_b, v01.x, ob[0]);
-          ob[1] = fmaf(pk_b, v01.y, ob[1]);
-          ob[2] = fmaf(pk_b, v23.x, ob[2]);
-          ob[3] = fmaf(pk_b, v23.y, ob[3]);
+    }
+    __syncthreads();
+    // ---- P.V over this warp's 8 keys, for every row
+    const uint8_t* vbase = st + C::TILE + pregion * C::KREG + (lane & 1) * 8;
+#pragma unroll
+    for (int r = 0; r < RM; ++r) {
+      if (r < R) {
+        const float al = srow[r];
+        acc[r][0] *= al; acc[r][1] *= al; acc[r][2] *= al; acc[r][3] *= al;
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int k = 8 * warp + kk;
+      const uint2 w = *reinterpret_cast<const uint2*>(vbase + k * 128 + ((pc ^ (k & 7)) << 4));
+      const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+      const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+#pragma unroll
+      for (int r = 0; r < RM; ++r) {
+        if (r < R) {
+          const float p = ss[r * C::KT + k];
+          acc[r][0] = fmaf(p, v01.x, acc[r][0]);
+          acc[r][1] = fmaf(p, v01.y, acc[r][1]);
+          acc[r][2] = fmaf(p, v23.x, acc[r][2]);
+          acc[r][3] = fmaf(p, v23.y, acc[r][3]);
         }
       }
     }
-    __syncthreads();                       // stage t % 2 is free again
+    __syncthreads();                       // stage t % 2 and the score rows are free again
     if (tid == 0 && t + 2 < n_tiles) issue(t + 2);
   }
   if (!ok) {
@@ -238,17 +255,40 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         mbar_wait_quiet(b_full0 + 8 * (t & 1), (t >> 1) & 1, 200000000ull);
     return;
   }
-  // the split's normalised partial and its lse
-  auto store = [&](int r, float m, float l, const float* o) {
+  // ---- sum the warps' partial O (in the query buffer, which is no longer needed), then normalise
+  for (int idx = tid; idx < C::R_MAX * D; idx += C::THREADS) sq[idx] = 0.f;
+  if (lane == 0) {
+    if (ra < R) srow[ra] = l_a;
+    if (rb < R) srow[rb] = l_b;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < RM; ++r) {
+    if (r < R) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) atomicAdd(sq + r * D + 4 * lane + e, acc[r][e]);
+    }
+  }
+  __syncthreads();
+  // thread = (row, 16-byte group of columns) writes the split's normalised partial
+  for (int idx = tid; idx < R * (D / 4); idx += C::THREADS) {
+    const int r = idx / (D / 4), c4 = idx % (D / 4);
     const int hq = bhq0 + r / a.Lq, i = r % a.Lq;
     const size_t row = (static_cast<size_t>(split) * a.bh + hq) * a.Lq + i;
+    const float l = srow[r];
     const float inv = l > 0.f ? 1.0f / l : 0.f;
-    *reinterpret_cast<float4*>(a.part_o + row * D + 4 * lane) = make_float4(o[0] * inv, o[1] * inv, o[2] * inv,
-                                                                           o[3] * inv);
-    if (lane == 0) a.part_lse[row] = l > 0.f ? (m * c2 + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-  };
-  if (va) store(ra, m_a, l_a, oa);
-  if (vb) store(rb, m_b, l_b, ob);
+    const float4 v = *reinterpret_cast<const float4*>(sq + r * D + 4 * c4);
+    *reinterpret_cast<float4*>(a.part_o + row * D + 4 * c4) = make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+  }
+  if (lane == 0) {
+    auto put_lse = [&](int r, float m, float l) {
+      const int hq = bhq0 + r / a.Lq, i = r % a.Lq;
+      const size_t row = (static_cast<size_t>(split) * a.bh + hq) * a.Lq + i;
+      a.part_lse[row] = l > 0.f ? (m * c2 + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    };
+    if (ra < R) put_lse(ra, m_a, l_a);
+    if (rb < R) put_lse(rb, m_b, l_b);
+  }
 }
 
 // One warp per query row: lse = ln sum_s e^{lse_s}, O = sum_s e^{lse_s - lse} O_s.

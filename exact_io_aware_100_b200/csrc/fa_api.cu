@@ -430,8 +430,12 @@ fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float*
   DevState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
   if (!ds->dec_attr) {
-    if (cudaFuncSetAttribute(fa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg::SMEM_BYTES) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(fa_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg::SMEM_BYTES) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fa_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg::SMEM_BYTES) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fa_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg::SMEM_BYTES) !=
+            cudaSuccess)
       return FA_ERR_CUDA;
     ds->dec_attr = true;
   }
@@ -458,7 +462,14 @@ fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float*
   a.part_o = reinterpret_cast<float*>(w);
   a.part_lse = reinterpret_cast<float*>(w + round256(static_cast<size_t>(a.n_splits) * rows * d * 4));
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  fa_decode_kernel<<<dim3(a.n_splits, a.bh_kv), DecCfg::THREADS, DecCfg::SMEM_BYTES, s>>>(tk, tv, a);
+  const dim3 grid(a.n_splits, a.bh_kv);
+  const int rows_per_set = a.group * Lq;
+  if (rows_per_set <= 4)
+    fa_decode_kernel<4><<<grid, DecCfg::THREADS, DecCfg::SMEM_BYTES, s>>>(tk, tv, a);
+  else if (rows_per_set <= 8)
+    fa_decode_kernel<8><<<grid, DecCfg::THREADS, DecCfg::SMEM_BYTES, s>>>(tk, tv, a);
+  else
+    fa_decode_kernel<16><<<grid, DecCfg::THREADS, DecCfg::SMEM_BYTES, s>>>(tk, tv, a);
   const size_t warps = rows, per_block = 8;
   size_t blocks = (warps + per_block - 1) / per_block;
   if (blocks > static_cast<size_t>(ds->sms) * 16) blocks = static_cast<size_t>(ds->sms) * 16;

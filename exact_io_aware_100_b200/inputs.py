@@ -39,6 +39,7 @@ class Workload:
     seed: int
     backward: bool = False
     h_kv: int = 0       # key/value heads (0: as many as query heads)
+    lq: int = 0         # decoding: this many query positions against N cached keys (0: N queries)
 
     @property
     def kv_heads(self) -> int:
@@ -49,6 +50,10 @@ class Workload:
         return 1.0 / math.sqrt(self.d)
 
     def fwd_flops(self) -> float:
+        if self.lq:
+            # query i of the last lq positions sees N - lq + i + 1 keys when causal, all N otherwise
+            keys = (self.lq * (self.N - self.lq) + self.lq * (self.lq + 1) // 2) if self.causal else self.lq * self.N
+            return 4.0 * self.B * self.H * keys * self.d
         f = 4.0 * self.B * self.H * self.N * self.N * self.d
         return f / 2 if self.causal else f
 
@@ -62,6 +67,8 @@ WORKLOADS = {
     "backward": Workload("backward", 4, 16, 4096, 128, True, "bf16", 1.0, 1005, True),
     # grouped-query attention on the prefill shape: 32 query heads over 8 key/value heads
     "prefill_gqa": Workload("prefill_gqa", 2, 32, 8192, 128, True, "bf16", 2.0, 1006, False, 8),
+    # decoding one token per sequence against an 8192-key cache, 32 query heads over 8 key/value heads
+    "decode": Workload("decode", 16, 32, 8192, 128, True, "bf16", 1.0, 1007, False, 8, 1),
 }
 
 
