@@ -119,8 +119,9 @@ __global__ void fa_bwd_dq_kernel(const BwdArgs a) {
 }
 
 // ------------------------------------------------------------------ main
+template <int D_>
 struct BwdCfg {
-  static constexpr int D = 128;
+  static constexpr int D = D_;                 // head dim, 64 or 128
   static constexpr int BN = 128;               // keys per CTA
   static constexpr int BM = 128;               // queries per iteration
   static constexpr int THREADS = 448;          // warps 0-7 P/dS, 8-11 dQ drain, 12 MMA, 13 TMA
@@ -134,32 +135,37 @@ struct BwdCfg {
   static constexpr int LAUNCH_REGS = 128;
   static constexpr int REGS_PDS = 144, REGS_DRAIN = 80, REGS_SINGLE = 112;
   static constexpr int REG = 128 * 128;        // one 64-column SW128 region of a 128-row bf16 tile
-  static constexpr int TILE = 2 * REG;         // a 128 x 128 bf16 tile (32 KB)
+  static constexpr int N_REG = D / 64;         // regions of a 128-row, D-column tile
+  static constexpr int TILE = N_REG * REG;     // a 128 x D bf16 tile (K, V, Q or dO)
+  static constexpr int DS_BYTES = 2 * REG;     // the 128 x 128 dS tile
   static constexpr int OFF_K = 0, OFF_V = TILE;
   static constexpr int OFF_Q = 2 * TILE;       // two Q stages
   static constexpr int OFF_DO = 4 * TILE;      // two dO stages
   static constexpr int OFF_PS = 6 * TILE;      // dS_i, stored [key][query]
-  static constexpr int OFF_VEC = 7 * TILE;     // per Q stage: lse2[BM] then D[BM]
+  static constexpr int OFF_VEC = OFF_PS + DS_BYTES;   // per Q stage: lse2[BM] then D[BM]
   static constexpr int VEC_BYTES = 2 * BM * 4;
   static constexpr int OFF_BAR = OFF_VEC + 2 * VEC_BYTES;
   static constexpr int N_BARS = 20;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int USED = OFF_MISC + 16;
-  // The opt-in maximum per block.  The kernel rounds its base up to 1 KB (SW128
-  // tiles) inside this and checks that USED still fits.
-  static constexpr int SMEM_BYTES = 232448;
+  // At most the opt-in maximum per block.  The kernel rounds its base up to 1 KB
+  // (SW128 tiles) inside this and checks that USED still fits.
+  static constexpr int SMEM_BYTES = (USED + 1024 < 232448) ? USED + 1024 : 232448;
   static constexpr uint32_t TMEM_COLS = 512;
-  // X: S^T, then dP^T.  Y: P^T (bf16, columns 0-63), then dQ^T (fp32, 128 columns)
-  static constexpr uint32_t T_DV = 0, T_DK = 128, T_X = 256, T_Y = 384;
+  // X: S^T, then dP^T.  Y: P^T (bf16, columns 0-63), then dQ^T (fp32, 128 columns;
+  // with D = 64 the MMA still writes 128 rows of dQ^T, of which lanes >= 64 read
+  // the tile after K and are never drained)
+  static constexpr uint32_t T_DV = 0, T_DK = D, T_X = 2 * D, T_Y = 2 * D + 128;
   static constexpr uint32_t IDESC_SD = idesc_bf16_f32(128, BM, false, false);   // S^T, dP^T
   static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);     // dV (A in TMEM), dK
   static constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, BM, true, true);      // dQ^T
 };
-static_assert(BwdCfg::USED + 768 <= BwdCfg::SMEM_BYTES, "shared memory plan");
-static_assert(BwdCfg::PDS_THREADS * BwdCfg::REGS_PDS + BwdCfg::DRAIN_THREADS * BwdCfg::REGS_DRAIN +
-                  64 * BwdCfg::REGS_SINGLE <= BwdCfg::THREADS * BwdCfg::LAUNCH_REGS,
+static_assert(BwdCfg<128>::USED + 768 <= BwdCfg<128>::SMEM_BYTES, "shared memory plan");
+static_assert(BwdCfg<64>::USED + 768 <= BwdCfg<64>::SMEM_BYTES, "shared memory plan");
+static_assert(BwdCfg<128>::PDS_THREADS * BwdCfg<128>::REGS_PDS + BwdCfg<128>::DRAIN_THREADS * BwdCfg<128>::REGS_DRAIN +
+                  64 * BwdCfg<128>::REGS_SINGLE <= BwdCfg<128>::THREADS * BwdCfg<128>::LAUNCH_REGS,
               "register split exceeds the registers the block launches with");
-static_assert(2 * BwdCfg::REGS_PDS + BwdCfg::REGS_DRAIN + BwdCfg::REGS_SINGLE <= 512,
+static_assert(2 * BwdCfg<128>::REGS_PDS + BwdCfg<128>::REGS_DRAIN + BwdCfg<128>::REGS_SINGLE <= 512,
               "register split exceeds a sub-partition");
 
 // Work item x -> (head, key block).  Heads are taken in groups of
@@ -176,11 +182,12 @@ __device__ __forceinline__ void bwd_decode(const BwdArgs& a, int x, int& bh, int
   bh = h0 + (r - kb * gh);
 }
 
-__global__ void __launch_bounds__(BwdCfg::THREADS, 1)
+template <int D_>
+__global__ void __launch_bounds__(BwdCfg<D_>::THREADS, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const BwdArgs args) {
-  using C = BwdCfg;
+  using C = BwdCfg<D_>;
   constexpr int D = C::D;
   extern __shared__ __align__(16) uint8_t smem_raw[];   // only 16 B promised: the 1 KB rounding below is real
   const uint32_t raw = smem_u32(smem_raw);
@@ -272,7 +279,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       bool ok = true;
       int q_last[2] = {-1, -1}, do_last[2] = {-1, -1};     // last query block loaded into each stage
       mbar_expect_tx(b_kv_full, 2 * C::TILE);
-      for (int r = 0; r < 2; ++r) {
+      for (int r = 0; r < C::N_REG; ++r) {
         tma_load_3d(sK + r * C::REG, &tm_k, b_kv_full, r * 64, k0, bh);
         tma_load_3d(sV + r * C::REG, &tm_v, b_kv_full, r * 64, k0, bh);
       }
@@ -284,7 +291,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // Q_i with its lse2 and D rows; the stage is released after dK_i
         if (round > 0 && !mbar_wait(b_q_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
         mbar_expect_tx(b_q_full(s), C::TILE + C::VEC_BYTES);
-        for (int r = 0; r < 2; ++r) tma_load_3d(sQ(s) + r * C::REG, &tm_q, b_q_full(s), r * 64, q0, hq);
+        for (int r = 0; r < C::N_REG; ++r) tma_load_3d(sQ(s) + r * C::REG, &tm_q, b_q_full(s), r * 64, q0, hq);
         const size_t voff = static_cast<size_t>(hq) * args.Np + q0;
         bulk_load(sVec(s), args.lse2 + voff, C::BM * 4, b_q_full(s));
         bulk_load(sVec(s) + C::BM * 4, args.dvec + voff, C::BM * 4, b_q_full(s));
@@ -292,7 +299,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // dO_i; the stage is released after dV_i
         if (round > 0 && !mbar_wait(b_do_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
         mbar_expect_tx(b_do_full(s), C::TILE);
-        for (int r = 0; r < 2; ++r) tma_load_3d(sDO(s) + r * C::REG, &tm_do, b_do_full(s), r * 64, q0, hq);
+        for (int r = 0; r < C::N_REG; ++r) tma_load_3d(sDO(s) + r * C::REG, &tm_do, b_do_full(s), r * 64, q0, hq);
         do_last[s] = it;
       }
       if (!ok) {       // let the loads in flight land before the CTA exits
@@ -496,17 +503,17 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       fence_proxy_async_smem();
       mbar_arrive(b_ds_ready);
     }
-    // ---- epilogue: this thread's half of the dV, dK rows -> global
+    // ---- epilogue: this thread's half of the dV, dK rows (D / 2 columns) -> global
     if (ok && mbar_wait_warp(b_dkv_done, 0, ctl)) {
       tc_fence_after();
-      const size_t grow = (static_cast<size_t>(bh) * args.N + key) * D + 64 * ch;
+      const size_t grow = (static_cast<size_t>(bh) * args.N + key) * D + (D / 2) * ch;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DK : C::T_DV) + 64 * ch;
+        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DK : C::T_DV) + (D / 2) * ch;
         __nv_bfloat16* dst = (which ? args.dk : args.dv) + grow;
         const float mul = which ? args.scale : 1.0f;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t v[32];
           tmem_ld32(tsrc + c * 32, v);
           tmem_wait_ld();
@@ -548,7 +555,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         mbar_arrive(h == 0 ? b_ylo_free : b_yhi_free);
         float* a_row = acc + static_cast<size_t>(q0 + 64 * h) * D;
-        const int nh = nq - 64 * h;      // valid rows in this half (may be <= 0)
+        // valid rows in this half (may be <= 0); none for the lanes past the head dim (D = 64)
+        const int nh = dl < D ? nq - 64 * h : 0;
         if (nh >= 64) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) red_add_f32(a_row + static_cast<size_t>(c) * D, __uint_as_float(r[c]));

@@ -26,7 +26,7 @@ struct DevState {
   bool ready = false;
   uint32_t* status = nullptr;
   int sms = 0;
-  bool fwd_attr64 = false, fwd_attr128 = false, bwd_attr = false, dec_attr = false;
+  bool fwd_attr64 = false, fwd_attr128 = false, bwd_attr64 = false, bwd_attr128 = false, dec_attr = false;
 };
 DevState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -244,6 +244,17 @@ namespace {
 
 enum BwdPhase : int { PH_PREPARE = 1, PH_MAIN = 2, PH_FINISH = 4, PH_ALL = 7 };
 
+// First use of the backward main kernel for head dim D on a device.
+template <int D>
+fa_status prepare_bwd_kernel() {
+  using C = BwdCfg<D>;
+  if (!launch_regs_are(reinterpret_cast<const void*>(fa_bwd_kernel<D>), C::LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(fa_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 // Validates, fills the kernel arguments, and launches the requested phases.
 fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dout, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
@@ -251,7 +262,7 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   fa_status st = check_sizes(B, H, N, d, scale);
   if (st != FA_OK) return st;
   if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if ((phases & PH_PREPARE) && (!aligned16(o) || !aligned16(lse) || !aligned16(dout))) return FA_ERR_ALIGN;
   if ((phases & PH_MAIN) && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
                              !aligned16(dk) || !aligned16(dv)))
@@ -262,13 +273,10 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
     return FA_ERR_WORKSPACE;
   DevState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
-  using C = BwdCfg;
-  if ((phases & PH_MAIN) && !ds->bwd_attr) {
-    if (!launch_regs_are(reinterpret_cast<const void*>(fa_bwd_kernel), C::LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(fa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return FA_ERR_CUDA;
-    ds->bwd_attr = true;
+  if ((phases & PH_MAIN) && !(d == 64 ? ds->bwd_attr64 : ds->bwd_attr128)) {
+    st = d == 64 ? prepare_bwd_kernel<64>() : prepare_bwd_kernel<128>();
+    if (st != FA_OK) return st;
+    (d == 64 ? ds->bwd_attr64 : ds->bwd_attr128) = true;
   }
   const int BH = B * H;
   BwdArgs a;
@@ -299,15 +307,29 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.wait_limit_ns = kWaitLimitNs;
-  if (phases & PH_PREPARE) fa_bwd_pre_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
+  if (phases & PH_PREPARE) {
+    if (d == 64)
+      fa_bwd_pre_kernel<64><<<ds->sms * 8, 256, 0, stream>>>(a);
+    else
+      fa_bwd_pre_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
+  }
   if (phases & PH_MAIN) {
     CUtensorMap tq, tk, tv, tdo;
     if (!make_map(&tq, q, d, N, BH, 128) || !make_map(&tk, k, d, N, a.bh_kv, 128) ||
         !make_map(&tv, v, d, N, a.bh_kv, 128) || !make_map(&tdo, dout, d, N, BH, 128))
       return FA_ERR_CUDA;
-    fa_bwd_kernel<<<a.n_kb * a.bh_kv, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    if (d == 64)
+      fa_bwd_kernel<64><<<a.n_kb * a.bh_kv, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+    else
+      fa_bwd_kernel<128><<<a.n_kb * a.bh_kv, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo,
+                                                                                                       a);
   }
-  if (phases & PH_FINISH) fa_bwd_dq_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
+  if (phases & PH_FINISH) {
+    if (d == 64)
+      fa_bwd_dq_kernel<64><<<ds->sms * 8, 256, 0, stream>>>(a);
+    else
+      fa_bwd_dq_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
+  }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

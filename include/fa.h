@@ -28,7 +28,8 @@
  *    anything is launched.  A kernel whose internal wait gives up (a bug, or a
  *    device that stopped making progress) sets a device status word that
  *    fa_get_device_status() reports; outputs are then undefined.
- *  - Supported: d in {64, 128} for the forward, d == 128 for the backward;
+ *  - Supported: d in {64, 128} for the forward and the backward (d == 128 for
+ *    fa_decode);
  *    1 <= N <= 2^24; B*H*N*d < 2^31 elements per tensor.
  */
 #ifndef FA_H
@@ -83,7 +84,7 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
 size_t fa_fwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype);
 
 /*
- * Backward, bf16, d == 128.  Inputs q, k, v, o, dO: [B,H,N,d] bf16; lse from the
+ * Backward, bf16, d in {64, 128}.  Inputs q, k, v, o, dO: [B,H,N,d] bf16; lse from the
  * forward: [B,H,N] float.  Outputs dq, dk, dv: [B,H,N,d] bf16 (written, not
  * accumulated).  workspace: device memory of at least fa_bwd_workspace_size()
  * bytes, 256-byte aligned (holds the fp32 dQ accumulator and per-row D, lse).
@@ -128,7 +129,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *  lse: [B,H,N] float.  dk and dv of a shared head are the sums over its set.
  * Same layout, ownership, alignment, stream and error rules as fa_fwd /
  * fa_bwd, plus FA_ERR_INVALID when H_kv < 1 or H is not a multiple of H_kv.
- * fa_bwd_gqa needs d == 128 and fa_bwd_workspace_size(B, H, N, d) bytes of
+ * fa_bwd_gqa takes d in {64, 128} and fa_bwd_workspace_size(B, H, N, d) bytes of
  * workspace (sized by the query heads).
  */
 fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -66,7 +66,7 @@ def test_argument_validation_without_device(lib):
     assert g(P16, P16, P16, P16, P16, 1, 1, 128, 64, 0.125, 0, 7, None, 0, None) == 2
     b = lib.fa_bwd
     args = [P16] * 9
-    assert b(*args, 1, 1, 128, 64, 0.125, 1, P16, 1 << 30, None) == 2              # bwd d=64
+    assert b(*args, 1, 1, 128, 96, 0.125, 1, P16, 1 << 30, None) == 2              # bwd d=96
     assert b(*args, 1, 1, 128, 128, 0.125, 1, None, 0, None) == 4                  # no workspace
     need = lib.fa_bwd_workspace_size(1, 1, 128, 128)
     assert b(*args, 1, 1, 128, 128, 0.125, 1, 256, need - 1, None) == 4           # too small
@@ -81,7 +81,7 @@ def test_grouped_query_validation_without_device(lib):
     assert f(P16, P16, P16, P16, P16 + 4, 1, 6, 2, 128, 64, 0.125, 0, None) == 3  # misaligned
     args = [P16] * 9
     assert b(*args, 1, 6, 4, 128, 128, 0.125, 1, P16, 1 << 30, None) == 1         # uneven sets
-    assert b(*args, 1, 6, 3, 128, 64, 0.125, 1, P16, 1 << 30, None) == 2          # d = 64
+    assert b(*args, 1, 6, 3, 128, 96, 0.125, 1, P16, 1 << 30, None) == 2          # d = 96
     assert b(*args, 1, 6, 3, 128, 128, 0.125, 1, None, 0, None) == 4              # no workspace
 
 

@@ -53,6 +53,23 @@ def test_backward_ragged(N, causal):
     check_heads(host, dq, dk, dv, range(B * H), H, causal, 1.0 / np.sqrt(d))
 
 
+@pytest.mark.parametrize("N", [1, 100, 129, 300, 640])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_head_dim_64(N, causal):
+    B, H, d = 2, 3, 64
+    host, _ = make_case(B, H, N, d, 9300 + N, names=("q", "k", "v", "do"))
+    dq, dk, dv = run_bwd(host, causal)
+    check_heads(host, dq, dk, dv, range(B * H), H, causal, 1.0 / np.sqrt(d))
+
+
+def test_backward_multi_head_shape_head_dim_64():
+    """The multi-head configuration's sizes (B=4 H=16 N=2048, d = 64) on sampled heads."""
+    B, H, N, d = 4, 16, 2048, 64
+    host, _ = make_case(B, H, N, d, 9400, names=("q", "k", "v", "do"))
+    dq, dk, dv = run_bwd(host, True)
+    check_heads(host, dq, dk, dv, [0, 21, 42, 63], H, True, 1.0 / np.sqrt(d))
+
+
 def test_backward_many_heads_and_sharp_rows():
     B, H, N, d = 3, 7, 320, 128
     host, _ = make_case(B, H, N, d, 9100, k_scale=4.0, names=("q", "k", "v", "do"))

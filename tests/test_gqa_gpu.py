@@ -47,16 +47,17 @@ def test_gqa_forward_matches_oracle(B, H, H_kv, N, d, causal):
     assert_lse(to_f64(lse), rl)
 
 
-@pytest.mark.parametrize("B,H,H_kv,N,causal", [
-    (1, 4, 2, 300, True),
-    (1, 4, 2, 257, False),
-    (2, 3, 1, 200, True),           # multi-query
-    (1, 8, 2, 640, True),
+@pytest.mark.parametrize("B,H,H_kv,N,causal,d", [
+    (1, 4, 2, 300, True, 128),
+    (1, 4, 2, 257, False, 128),
+    (2, 3, 1, 200, True, 128),      # multi-query
+    (1, 8, 2, 640, True, 128),
+    (1, 4, 2, 300, True, 64),
+    (2, 6, 1, 200, False, 64),
 ])
-def test_gqa_backward_matches_oracle(B, H, H_kv, N, causal):
+def test_gqa_backward_matches_oracle(B, H, H_kv, N, causal, d):
     import torch
     import exact_io_aware_100_b200 as fa
-    d = 128
     host, f64 = _case(B, H, H_kv, N, d, 2200 + H + N, ("q", "k", "v", "do"))
     q, k, v, do = (to_device(host[n], "bf16") for n in ("q", "k", "v", "do"))
     o, lse = fa.forward(q, k, v, causal)
