@@ -7,6 +7,10 @@ from .attention import (  # noqa: F401
     attention_fwd_gqa,
     attention_fwd_blockwise,
     attention_fwd_decode,
+    attention_fwd_general,
+    attention_bwd_general,
+    attention_fwd_varlen,
+    attention_bwd_varlen,
     attention_fwd_rows,
     softmax_merge,
 )

@@ -48,6 +48,16 @@ Readings where the pages are silent or garbled (each is listed in the design doc):
     key/value head but not which; the sets are contiguous, query head h using
     key/value head h // (H / H_kv), and a shared head's gradient is the sum of
     the gradients of its uses.
+  * any number of queries against any number of keys (the library interface
+    users of the integrations in [P5] "پیاده‌سازی و استفاده از Flash Attention"
+    expect; the pages define no variant): causal alignment stays bottom-right,
+    query i sees keys j <= N_k - N_q + i, so with N_q > N_k the first
+    N_q - N_k queries see no key at all.  A query that sees no key (also
+    N_k = 0) has O = 0 (the empty weighted sum) and lse = -inf (ln of an empty
+    sum); its gradient is zero;
+  * variable-length batches: sequence b is the packed rows cu_q[b]:cu_q[b+1]
+    of q [T_q, H, d] and cu_k[b]:cu_k[b+1] of k, v [T_k, H_kv, d]; each
+    sequence is its own attention problem; lse is stored [H, T_q].
 
 Parity pins for every function live in tests/test_oracle.py; none of the
 functions below is "parity unpinned".
@@ -64,6 +74,10 @@ __all__ = [
     "attention_fwd_gqa",
     "attention_bwd_gqa",
     "attention_fwd_decode",
+    "attention_fwd_general",
+    "attention_bwd_general",
+    "attention_fwd_varlen",
+    "attention_bwd_varlen",
     "softmax_merge",
     "attention_fwd_blockwise",
 ]
@@ -246,6 +260,121 @@ def attention_fwd_decode(q, k, v, scale: float, causal: bool):
             o[b, h] = p @ v[b, g]
             lse[b, h] = l_
     return o, lse
+
+
+def _attend(q, k, v, scale: float, causal: bool):
+    """One head of one sequence: N_q queries against N_k keys (either may be 0).
+
+    [P1] ``standard_attention`` with the bottom-right causal reading of the
+    module doc: S = scale Q K^T, s_ij = -inf for j > N_k - N_q + i; rows that
+    keep at least one key get the two-pass softmax; rows that keep none get
+    P = 0, O = 0, lse = -inf.  Returns (O [N_q, d_v], lse [N_q], P [N_q, N_k]).
+    """
+    nq, nk = q.shape[0], k.shape[0]
+    s = scale * (q @ k.T)
+    if causal:
+        last_key = np.arange(nq)[:, None] + (nk - nq)
+        s = np.where(np.arange(nk)[None, :] > last_key, -np.inf, s)
+    p = np.zeros((nq, nk))
+    lse = np.full(nq, -np.inf)
+    seen = np.isfinite(s).any(axis=1) if nk > 0 else np.zeros(nq, dtype=bool)
+    if seen.any():
+        p[seen], lse[seen] = _softmax_rows(s[seen])
+    return p @ v, lse, p
+
+
+def _attend_grad(q, k, v, do, p, scale: float):
+    """Exact gradients of one head of one sequence from its probabilities P
+    (same formulas as ``attention_bwd``; rows with P = 0 contribute nothing)."""
+    dv = p.T @ do
+    dp = do @ v.T
+    ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+    return scale * (ds @ k), scale * (ds.T @ q), dv
+
+
+def attention_fwd_general(q, k, v, scale: float, causal: bool):
+    """Forward for q [B, H, N_q, d] against k, v [B, H_kv, N_k, d], any N_q, N_k.
+
+    Grouped heads as in ``attention_fwd_gqa``; each (b, h) is ``_attend``.
+    Returns (O [B, H, N_q, d_v], lse [B, H, N_q]) in float64.
+    """
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    B, H, Nq, _ = q.shape
+    H_kv = k.shape[1]
+    o = np.empty((B, H, Nq, v.shape[-1]))
+    lse = np.empty((B, H, Nq))
+    for b in range(B):
+        for h in range(H):
+            g = _kv_head(h, H, H_kv)
+            o[b, h], lse[b, h], _ = _attend(q[b, h], k[b, g], v[b, g], scale, causal)
+    return o, lse
+
+
+def attention_bwd_general(q, k, v, do, scale: float, causal: bool):
+    """Exact gradients of sum(dO * O) for O = attention_fwd_general(...); a
+    shared key/value head sums the gradients of its uses."""
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    B, H = q.shape[:2]
+    H_kv = k.shape[1]
+    dq = np.empty_like(q)
+    dk, dv = np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            g = _kv_head(h, H, H_kv)
+            _, _, p = _attend(q[b, h], k[b, g], v[b, g], scale, causal)
+            dq[b, h], dk_h, dv_h = _attend_grad(q[b, h], k[b, g], v[b, g], do[b, h], p, scale)
+            dk[b, g] += dk_h
+            dv[b, g] += dv_h
+    return dq, dk, dv
+
+
+def _check_offsets(cu, total: int) -> np.ndarray:
+    cu = np.asarray(cu, dtype=np.int64)
+    if cu.ndim != 1 or cu.size < 1 or cu[0] != 0 or cu[-1] != total or np.any(np.diff(cu) < 0):
+        raise ValueError("sequence offsets must start at 0, never decrease and end at the row count")
+    return cu
+
+
+def attention_fwd_varlen(q, k, v, cu_q, cu_k, scale: float, causal: bool):
+    """Variable-length batch: q [T_q, H, d], k, v [T_k, H_kv, d] packed by sequence.
+
+    Sequence b is rows cu_q[b]:cu_q[b+1] of q against rows cu_k[b]:cu_k[b+1]
+    of k and v, each head by ``_attend``.  Returns (O [T_q, H, d_v],
+    lse [H, T_q]) in float64.
+    """
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    cu_q, cu_k = _check_offsets(cu_q, q.shape[0]), _check_offsets(cu_k, k.shape[0])
+    if cu_q.size != cu_k.size:
+        raise ValueError("query and key offsets describe different batch sizes")
+    H, H_kv = q.shape[1], k.shape[1]
+    o = np.zeros((q.shape[0], H, v.shape[-1]))
+    lse = np.full((H, q.shape[0]), -np.inf)
+    for b in range(cu_q.size - 1):
+        qs, ks = slice(cu_q[b], cu_q[b + 1]), slice(cu_k[b], cu_k[b + 1])
+        for h in range(H):
+            g = _kv_head(h, H, H_kv)
+            o[qs, h], lse[h, qs], _ = _attend(q[qs, h], k[ks, g], v[ks, g], scale, causal)
+    return o, lse
+
+
+def attention_bwd_varlen(q, k, v, do, cu_q, cu_k, scale: float, causal: bool):
+    """Exact gradients of sum(dO * O) for O = attention_fwd_varlen(...)."""
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    cu_q, cu_k = _check_offsets(cu_q, q.shape[0]), _check_offsets(cu_k, k.shape[0])
+    if cu_q.size != cu_k.size:
+        raise ValueError("query and key offsets describe different batch sizes")
+    H, H_kv = q.shape[1], k.shape[1]
+    dq = np.zeros_like(q)
+    dk, dv = np.zeros_like(k), np.zeros_like(v)
+    for b in range(cu_q.size - 1):
+        qs, ks = slice(cu_q[b], cu_q[b + 1]), slice(cu_k[b], cu_k[b + 1])
+        for h in range(H):
+            g = _kv_head(h, H, H_kv)
+            _, _, p = _attend(q[qs, h], k[ks, g], v[ks, g], scale, causal)
+            dq[qs, h], dk_h, dv_h = _attend_grad(q[qs, h], k[ks, g], v[ks, g], do[qs, h], p, scale)
+            dk[ks, g] += dk_h
+            dv[ks, g] += dv_h
+    return dq, dk, dv
 
 
 def softmax_merge(m_x, l_x, o_x, m_y, l_y, o_y):
