@@ -24,9 +24,23 @@ FA_BF16, FA_F32 = 0, 1
 EXPORTS = (
     "fa_fwd", "fa_fwd_ex", "fa_fwd_workspace_size", "fa_bwd", "fa_bwd_workspace_size",
     "fa_bwd_prepare", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc", "fa_fwd_gqa", "fa_bwd_gqa",
-    "fa_decode", "fa_decode_workspace_size",
+    "fa_decode", "fa_decode_workspace_size", "fa_fwd_general", "fa_bwd_general", "fa_bwd_general_workspace_size",
     "fa_get_device_status", "fa_selftest_wait_timeout", "fa_status_string", "fa_version",
 )
+
+
+class FaStrides(ctypes.Structure):
+    """fa_strides: element strides of one [batch][head][row][d] operand."""
+    _fields_ = [("batch", ctypes.c_int64), ("head", ctypes.c_int64), ("row", ctypes.c_int64)]
+
+
+class FaLayout(ctypes.Structure):
+    """fa_layout: sizes, packed-sequence offsets and operand strides (include/fa.h)."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int), ("d", ctypes.c_int),
+                ("Nq", ctypes.c_int), ("Nk", ctypes.c_int),
+                ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+                ("total_q", ctypes.c_int), ("total_k", ctypes.c_int)] + \
+               [(n, FaStrides) for n in ("q", "k", "v", "o", "dout", "dq", "dk", "dv")]
 
 
 class FaError(RuntimeError):
@@ -63,13 +77,19 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_decode_workspace_size.restype = Z
     L.fa_bwd_workspace_size.argtypes = [I, I, I, I]
     L.fa_bwd_workspace_size.restype = Z
+    LP = ctypes.POINTER(FaLayout)
+    L.fa_fwd_general.argtypes = [P, P, P, P, P, LP, F, I, P]
+    L.fa_bwd_general.argtypes = [P, P, P, P, P, P, P, P, P, LP, F, I, P, Z, P]
+    L.fa_bwd_general_workspace_size.argtypes = [LP]
+    L.fa_bwd_general_workspace_size.restype = Z
     L.fa_get_device_status.argtypes = [P]
     L.fa_selftest_wait_timeout.argtypes = [U64, P]
     L.fa_status_string.argtypes = [I]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_version.restype = ctypes.c_char_p
     for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_prepare", "fa_bwd_main", "fa_bwd_finish", "fa_bwd_noalloc",
-                 "fa_fwd_gqa", "fa_bwd_gqa", "fa_decode", "fa_get_device_status", "fa_selftest_wait_timeout"):
+                 "fa_fwd_gqa", "fa_bwd_gqa", "fa_decode", "fa_fwd_general", "fa_bwd_general",
+                 "fa_get_device_status", "fa_selftest_wait_timeout"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -233,6 +253,76 @@ def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
     return int(load_library().fa_bwd_workspace_size(B, H, N, d))
 
 
+# ----------------------------------------------------------------- general layouts
+def _strides_4d(t) -> FaStrides:
+    """Strides of a tensor viewed as [B, heads, rows, d] (d contiguous), any other strides."""
+    if t is None:
+        return FaStrides(0, 0, 0)
+    if t.dim() != 4 or (t.shape[3] > 1 and t.stride(3) != 1):
+        raise ValueError("expected a [B, heads, rows, d] tensor with contiguous d")
+    return FaStrides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _strides_packed(t) -> FaStrides:
+    """Strides of a packed [rows, heads, d] tensor (d contiguous)."""
+    if t is None:
+        return FaStrides(0, 0, 0)
+    if t.dim() != 3 or (t.shape[2] > 1 and t.stride(2) != 1):
+        raise ValueError("expected a packed [rows, heads, d] tensor with contiguous d")
+    return FaStrides(0, t.stride(1), t.stride(0))
+
+
+def layout_4d(q, k, v, o, dout=None, dq=None, dk=None, dv=None) -> FaLayout:
+    """fa_layout for fixed lengths: q, o, dout, dq [B, H, Nq, d] and k, v, dk, dv [B, H_kv, Nk, d],
+    as tensors of any strides (a [B, N, H, d] tensor is passed as its transpose(1, 2))."""
+    B, H, Nq, d = q.shape
+    Nk, H_kv = k.shape[2], k.shape[1]
+    L = FaLayout(B=B, H=H, H_kv=H_kv, d=d, Nq=Nq, Nk=Nk, cu_seqlens_q=None, cu_seqlens_k=None, total_q=0,
+                 total_k=0)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        setattr(L, name, _strides_4d(t))
+    return L
+
+
+def layout_packed(q, k, v, o, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                  dout=None, dq=None, dk=None, dv=None) -> FaLayout:
+    """fa_layout for packed sequences: q, o [total_q, H, d]; k, v [total_k, H_kv, d]; cu_seqlens_*
+    int32 device tensors of B + 1 row offsets; max_seqlen_* at least every sequence's length."""
+    total_q, H, d = q.shape
+    total_k, H_kv = k.shape[0], k.shape[1]
+    for cu in (cu_seqlens_q, cu_seqlens_k):
+        import torch
+        if cu.dtype != torch.int32 or cu.dim() != 1 or not cu.is_contiguous():
+            raise ValueError("sequence offsets must be a contiguous 1-D int32 tensor")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("query and key offsets must both hold B + 1 entries")
+    L = FaLayout(B=cu_seqlens_q.numel() - 1, H=H, H_kv=H_kv, d=d, Nq=int(max_seqlen_q), Nk=int(max_seqlen_k),
+                 cu_seqlens_q=cu_seqlens_q.data_ptr(), cu_seqlens_k=cu_seqlens_k.data_ptr(),
+                 total_q=total_q, total_k=total_k)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        setattr(L, name, _strides_packed(t))
+    return L
+
+
+def fa_fwd_general(q, k, v, o, lse, layout: FaLayout, causal: bool, scale: float | None = None,
+                   stream=None) -> None:
+    scale = 1.0 / math.sqrt(layout.d) if scale is None else float(scale)
+    _check(load_library().fa_fwd_general(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(layout),
+                                         scale, int(bool(causal)), _stream(stream)), "fa_fwd_general")
+
+
+def fa_bwd_general(q, k, v, o, lse, dout, dq, dk, dv, layout: FaLayout, causal: bool, workspace,
+                   scale: float | None = None, stream=None) -> None:
+    scale = 1.0 / math.sqrt(layout.d) if scale is None else float(scale)
+    _check(load_library().fa_bwd_general(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                                         _ptr(dk), _ptr(dv), ctypes.byref(layout), scale, int(bool(causal)),
+                                         _ptr(workspace), _ws_bytes(workspace), _stream(stream)), "fa_bwd_general")
+
+
+def fa_bwd_general_workspace_size(layout: FaLayout) -> int:
+    return int(load_library().fa_bwd_general_workspace_size(ctypes.byref(layout)))
+
+
 def fa_get_device_status(stream=None) -> int:
     return int(load_library().fa_get_device_status(_stream(stream)))
 
@@ -250,10 +340,24 @@ def _workspace(nbytes: int, device):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
+def _is_dense(*ts) -> bool:
+    return all(t.dim() == 4 and t.is_contiguous() for t in ts)
+
+
 def forward(q, k, v, causal: bool, scale: float | None = None, stream=None):
-    """O, lse for q [B,H,N,d] and k, v [B,H_kv,N,d] (bf16; float32 via the bf16 tensor-core path when
-    H_kv == H).  H_kv < H is grouped-query attention (contiguous sets of H / H_kv query heads)."""
+    """O, lse for q [B,H,Nq,d] and k, v [B,H_kv,Nk,d] (bf16; float32 via the bf16 tensor-core path when
+    the tensors are dense, H_kv == H and Nq == Nk).  H_kv < H is grouped-query attention (contiguous sets
+    of H / H_kv query heads); Nq != Nk aligns the causal mask bottom-right.  The tensors may have any
+    strides with d contiguous (e.g. a [B, N, H, d] tensor passed as its transpose(1, 2)); O comes back
+    with q's strides."""
     import torch
+    if q.dtype == torch.bfloat16 and (not _is_dense(q, k, v) or q.shape[2] != k.shape[2]):
+        o = torch.empty_like(q)    # q's strides when q is dense in some order, else contiguous
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        fa_fwd_general(q, k, v, o, lse, layout_4d(q, k, v, o), causal, scale, stream)
+        return o, lse
+    if q.shape[2] != k.shape[2]:
+        raise ValueError("query and key lengths differ: bf16 inputs only")
     B, H, N, d = _bhnd(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
@@ -269,10 +373,23 @@ def forward(q, k, v, causal: bool, scale: float | None = None, stream=None):
     return o, lse
 
 
+def _like(t):
+    import torch
+    return torch.empty_like(t)     # t's strides when t is dense in some order, else contiguous
+
+
 def backward(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, stream=None, workspace=None):
     """dQ, dK, dV (bf16) from the forward's O and lse; dK, dV have k's head count (grouped-query
-    attention sums each shared head's gradient over its set)."""
+    attention sums each shared head's gradient over its set).  Any strides and Nq != Nk as in
+    ``forward``; the gradients come back with the strides of q, k, v."""
     import torch
+    if not _is_dense(q, k, v, o, dout) or q.shape[2] != k.shape[2]:
+        dq, dk, dv = _like(q), _like(k), _like(v)
+        L = layout_4d(q, k, v, o, dout, dq, dk, dv)
+        if workspace is None:
+            workspace = _workspace(fa_bwd_general_workspace_size(L), q.device)
+        fa_bwd_general(q, k, v, o, lse, dout, dq, dk, dv, L, causal, workspace, scale, stream)
+        return dq, dk, dv
     B, H, N, d = _bhnd(q)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
@@ -281,4 +398,28 @@ def backward(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, st
         fa_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, causal, workspace, scale, stream)
     else:
         fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal, workspace, scale, stream)
+    return dq, dk, dv
+
+
+def forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int, causal: bool,
+                   scale: float | None = None, stream=None):
+    """Packed variable-length batch (bf16): q [total_q, H, d], k, v [total_k, H_kv, d]; sequence b is rows
+    cu_seqlens_q[b]:cu_seqlens_q[b+1] (int32 device offsets).  Returns O [total_q, H, d] and
+    lse [H, total_q]; bottom-right causal alignment per sequence."""
+    import torch
+    o = _like(q)
+    lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    L = layout_packed(q, k, v, o, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k)
+    fa_fwd_general(q, k, v, o, lse, L, causal, scale, stream)
+    return o, lse
+
+
+def backward_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                    causal: bool, scale: float | None = None, stream=None, workspace=None):
+    """dQ, dK, dV of ``forward_varlen`` (packed like q, k, v)."""
+    dq, dk, dv = _like(q), _like(k), _like(v)
+    L = layout_packed(q, k, v, o, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dout, dq, dk, dv)
+    if workspace is None:
+        workspace = _workspace(fa_bwd_general_workspace_size(L), q.device)
+    fa_bwd_general(q, k, v, o, lse, dout, dq, dk, dv, L, causal, workspace, scale, stream)
     return dq, dk, dv

@@ -32,8 +32,11 @@
 //                         a warpgroup with one thread per head-dim lane drains
 //                         dQ^T into the fp32 dQ accumulator with atomic adds;
 //  * fa_bwd_dq_kernel:    dQ = bf16(scale * dQacc).
+// Sequences, lengths and strides follow layout.cuh (fixed or packed variable
+// lengths, bottom-right causal alignment, any row / head / batch strides).
 #pragma once
 
+#include "layout.cuh"
 #include "ptx.cuh"
 
 namespace fa {
@@ -41,20 +44,22 @@ namespace fa {
 struct BwdArgs {
   const __nv_bfloat16* o;
   const __nv_bfloat16* dout;
-  const float* lse;       // [BH, N]
-  float* lse2;            // [BH, Np] workspace: lse * log2(e), +inf on padded rows
-  float* dvec;            // [BH, Np] workspace: D_i
-  float* dq_acc;          // [BH, N, D] workspace (fp32)
+  const float* lse;       // indexed by row_index
+  float* lse2;            // [B*H][Np] workspace: lse * log2(e), +inf on rows without a query or a key
+  float* dvec;            // [B*H][Np] workspace: D_i
+  float* dq_acc;          // [acc_rows][D] workspace (fp32), row row_index
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   uint32_t* status;
-  int N, Np, bh;          // Np = n_qb * 128; bh = B * H (query heads)
+  SeqLayout L;
+  Strides so, sdo, sdq, sdk, sdv;   // element strides of o, dO, dq, dk, dv
+  int dq_dense;           // dq is [B][H][Nq][D] dense with fixed lengths (a flat copy of the accumulator)
+  int Np;                 // ceil(L.Nq / 128) * 128
+  long long acc_rows;     // rows of the dQ accumulator: B*H*Nq, or H*total_q for packed sequences
   int bh_kv;              // B * H_kv (key/value heads); the main kernel's work items
-  int heads;              // H
   int group;              // query heads per key/value head
-  int n_kb;               // ceil(N / 128) key blocks
-  int n_qb;               // ceil(N / 128) query blocks
+  int n_kb;               // ceil(L.Nk / 128) key blocks
   int heads_per_group;    // work-item order of the main kernel
   int causal;
   float scale;
@@ -63,58 +68,128 @@ struct BwdArgs {
 };
 
 // ------------------------------------------------------------------ pre
-// One warp per query row: D_i = sum_c dO_ic O_ic (bf16 inputs, fp32 sum).
-template <int D>
-__global__ void fa_bwd_pre_kernel(const BwdArgs a) {
-  const int warps = (gridDim.x * blockDim.x) >> 5;
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const long long rows = static_cast<long long>(a.bh) * a.Np;
-  for (long long r = gw; r < rows; r += warps) {
-    const int bh = static_cast<int>(r / a.Np);
-    const int i = static_cast<int>(r % a.Np);
-    float acc = 0.f;
-    if (i < a.N) {
-      const size_t base = (static_cast<size_t>(bh) * a.N + i) * D;
-      constexpr int PER = D / 32;        // elements per lane
-      const __nv_bfloat16* po = a.o + base + lane * PER;
-      const __nv_bfloat16* pd = a.dout + base + lane * PER;
+// D_i = sum_c dO_ic O_ic (bf16 inputs, fp32 sum) and lse_i * log2(e), then the
+// fp32 dQ accumulator is zeroed.  HBM-bound: each lane reads 16-byte chunks (a
+// row is D / 8 lanes) and a warp keeps U passes of rows in flight before it
+// reduces them.
+__device__ __forceinline__ float dot_bf16x8(uint4 x, uint4 y) {
+  const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+  float acc = 0.f;
 #pragma unroll
-      for (int e = 0; e < PER; e += 2) {
-        const float2 fo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(po + e));
-        const float2 fd = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(pd + e));
-        acc = fmaf(fo.x, fd.x, acc);
-        acc = fmaf(fo.y, fd.y, acc);
+  for (int e = 0; e < 4; ++e) {
+    const float2 fx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[e]));
+    const float2 fy = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ys[e]));
+    acc = fmaf(fx.x, fy.x, acc);
+    acc = fmaf(fx.y, fy.y, acc);
+  }
+  return acc;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdArgs a) {
+  constexpr int CPR = D / 8;           // 16-byte chunks per row
+  constexpr int RPW = 32 / CPR;        // rows per warp per pass
+  constexpr int U = 4;                 // passes in flight
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / CPR, ch = lane % CPR;
+  const long long rows = static_cast<long long>(a.L.B) * a.L.H * a.Np;
+  const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long r0 = gw * (RPW * U); r0 < rows; r0 += nw * (RPW * U)) {   // warp-uniform loop
+    uint4 xo[U], xd[U];
+    float lv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long r = r0 + u * RPW + sub;
+      xo[u] = xd[u] = make_uint4(0u, 0u, 0u, 0u);
+      lv[u] = -INFINITY;
+      if (r < rows) {
+        const int bh = static_cast<int>(r / a.Np);
+        const int i = static_cast<int>(r - static_cast<long long>(bh) * a.Np);
+        const int b = bh / a.L.H, h = bh - b * a.L.H;
+        const SeqSpan sp = seq_span_any(a.L, b, a.status);
+        if (i < sp.nq) {
+          xo[u] = __ldg(reinterpret_cast<const uint4*>(a.o + row_offset(a.so, sp.bc, h, sp.q0 + i) + ch * 8));
+          xd[u] = __ldg(reinterpret_cast<const uint4*>(a.dout + row_offset(a.sdo, sp.bc, h, sp.q0 + i) + ch * 8));
+          if (ch == 0) lv[u] = a.lse[row_index_any(a.L, sp, h, i)];
+        }
       }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      a.dvec[r] = acc;
-      a.lse2[r] = (i < a.N) ? a.lse[static_cast<size_t>(bh) * a.N + i] * 1.4426950408889634f : INFINITY;
+    for (int u = 0; u < U; ++u) {
+      float acc = dot_bf16x8(xo[u], xd[u]);
+#pragma unroll
+      for (int off = CPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const long long r = r0 + u * RPW + sub;
+      if (ch == 0 && r < rows) {
+        // rows past the sequence end, and rows that see no key (lse = -inf), get
+        // +inf: their P = 2^(s - inf) is 0
+        a.dvec[r] = acc;
+        a.lse2[r] = lv[u] == -INFINITY ? INFINITY : lv[u] * 1.4426950408889634f;
+      }
     }
   }
   // zero the dQ accumulator
-  const size_t n4 = static_cast<size_t>(a.bh) * a.N * D / 4;
+  const size_t n4 = static_cast<size_t>(a.acc_rows) * D / 4;
   float4* q4 = reinterpret_cast<float4*>(a.dq_acc);
-  for (size_t k = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < n4;
-       k += static_cast<size_t>(gridDim.x) * blockDim.x)
-    q4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t k = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; k + 3 * stride < n4; k += 4 * stride) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) q4[k + u * stride] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (; k < n4; k += stride) q4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ------------------------------------------------------------------ dQ convert
+// dQ = bf16(scale * dQacc), four 16-byte loads in flight per thread.
+__device__ __forceinline__ uint2 scale_pack4(float4 v, float s) {
+  uint2 w;
+  w.x = pack_bf16x2(v.x * s, v.y * s);
+  w.y = pack_bf16x2(v.z * s, v.w * s);
+  return w;
+}
+
 template <int D>
-__global__ void fa_bwd_dq_kernel(const BwdArgs a) {
-  const size_t n4 = static_cast<size_t>(a.bh) * a.N * D / 4;
+__device__ __forceinline__ long long dq_offset(const BwdArgs& a, size_t k) {   // element of dq for float4 k
+  const long long ar = static_cast<long long>(k / (D / 4));
+  const int c = static_cast<int>(k % (D / 4)) * 4;
+  if (a.L.cu_q) {            // [H][total_q]: the row is the packed row coordinate
+    const int h = static_cast<int>(ar / a.L.total_q);
+    return row_offset(a.sdq, 0, h, static_cast<int>(ar - static_cast<long long>(h) * a.L.total_q)) + c;
+  }
+  const long long bh = ar / a.L.Nq;  // [B][H][Nq]
+  const int b = static_cast<int>(bh / a.L.H);
+  return row_offset(a.sdq, b, static_cast<int>(bh - static_cast<long long>(b) * a.L.H),
+                    static_cast<int>(ar - bh * a.L.Nq)) + c;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdArgs a) {
+  const size_t n4 = static_cast<size_t>(a.acc_rows) * D / 4;
   const float4* q4 = reinterpret_cast<const float4*>(a.dq_acc);
-  uint2* out = reinterpret_cast<uint2*>(a.dq);
-  for (size_t k = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < n4;
-       k += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const float4 v = q4[k];
-    uint2 w;
-    w.x = pack_bf16x2(v.x * a.scale, v.y * a.scale);
-    w.y = pack_bf16x2(v.z * a.scale, v.w * a.scale);
-    out[k] = w;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t k = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (a.dq_dense) {          // the accumulator's order is dq's
+    uint2* out = reinterpret_cast<uint2*>(a.dq);
+    for (; k + 3 * stride < n4; k += 4 * stride) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = q4[k + u * stride];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) out[k + u * stride] = scale_pack4(v[u], a.scale);
+    }
+    for (; k < n4; k += stride) out[k] = scale_pack4(q4[k], a.scale);
+  } else {                   // accumulator row -> (sequence, head, row) -> strided dq
+    for (; k + 3 * stride < n4; k += 4 * stride) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = q4[k + u * stride];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<uint2*>(a.dq + dq_offset<D>(a, k + u * stride)) = scale_pack4(v[u], a.scale);
+    }
+    for (; k < n4; k += stride) *reinterpret_cast<uint2*>(a.dq + dq_offset<D>(a, k)) = scale_pack4(q4[k], a.scale);
   }
 }
 
@@ -172,7 +247,7 @@ static_assert(2 * BwdCfg<128>::REGS_PDS + BwdCfg<128>::REGS_DRAIN + BwdCfg<128>:
 // heads_per_group; inside a group the key blocks with the most query blocks
 // come first (causal), so the dQ accumulators being added to at any time are
 // those of a few heads and stay in L2.
-__device__ __forceinline__ void bwd_decode(const BwdArgs& a, int x, int& bh, int& kb) {
+__device__ __forceinline__ void bwd_decode(const BwdArgs& a, int x, int& bh, int& kb) {   // bh: b * H_kv + h_kv
   const int per_group = a.heads_per_group * a.n_kb;
   const int g = x / per_group;
   const int r = x - g * per_group;
@@ -182,7 +257,7 @@ __device__ __forceinline__ void bwd_decode(const BwdArgs& a, int x, int& bh, int
   bh = h0 + (r - kb * gh);
 }
 
-template <int D_>
+template <int D_, bool PACKED>
 __global__ void __launch_bounds__(BwdCfg<D_>::THREADS, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -190,6 +265,30 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   using C = BwdCfg<D_>;
   constexpr int D = C::D;
   extern __shared__ __align__(16) uint8_t smem_raw[];   // only 16 B promised: the 1 KB rounding below is real
+  int bh, kb;                                        // bh: key/value head (b * H_kv + h_kv)
+  bwd_decode(args, static_cast<int>(blockIdx.x), bh, kb);
+  const int b = bh / args.L.H_kv, h_kv = bh - b * args.L.H_kv;
+  const SeqSpan sp = seq_span<PACKED>(args.L, b, args.status);
+  const int k0 = kb * C::BN;                         // first key of the block, in the sequence
+  if (k0 >= sp.nk) return;                           // past this sequence's keys: nothing to do
+  const int off = sp.nk - sp.nq;                     // bottom-right causal alignment
+  const int n_qb = (sp.nq + C::BM - 1) / C::BM;
+  // query blocks that see these keys (every key is seen by the last query row)
+  const int i_begin = args.causal ? max(0, k0 - off) / C::BM : 0;
+  const int n_per = max(0, n_qb - i_begin);          // per query head
+  const int n_iter = n_per * args.group;             // every query head of the set, one after the other
+  if (n_iter == 0) {                                 // no query at all: dK = dV = 0
+    const int nk = min(C::BN, sp.nk - k0);
+    for (int e = threadIdx.x; e < nk * (D / 8); e += blockDim.x) {
+      const int r = e / (D / 8), c = (e % (D / 8)) * 8;
+      *reinterpret_cast<uint4*>(args.dk + row_offset(args.sdk, sp.bc, h_kv, sp.k0 + k0 + r) + c) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(args.dv + row_offset(args.sdv, sp.bc, h_kv, sp.k0 + k0 + r) + c) = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
+  // query head (in the batch entry) and query block of iteration it
+  auto q_head = [&](int it) { return h_kv * args.group + it / n_per; };
+  auto q_row0 = [&](int it) { return (i_begin + it % n_per) * C::BM; };
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
   if (pad + C::USED > static_cast<uint32_t>(C::SMEM_BYTES)) {   // buffers do not fit: report, touch nothing
@@ -225,17 +324,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  int bh, kb;                                        // bh: key/value head
-  bwd_decode(args, static_cast<int>(blockIdx.x), bh, kb);
-  const int k0 = kb * C::BN;
-  const int i_begin = args.causal ? kb : 0;          // query blocks that see these keys (BM == BN)
-  const int n_per = args.n_qb - i_begin;             // per query head
-  const int n_iter = n_per * args.group;             // every query head of the set, one after the other
-  // query head and query block of iteration it
-  const int h_kv_count = args.heads / args.group;
-  const int bhq0 = (bh / h_kv_count) * args.heads + (bh % h_kv_count) * args.group;
-  auto q_head = [&](int it) { return bhq0 + it / n_per; };
-  auto q_row0 = [&](int it) { return (i_begin + it % n_per) * C::BM; };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0u;
@@ -280,8 +368,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       int q_last[2] = {-1, -1}, do_last[2] = {-1, -1};     // last query block loaded into each stage
       mbar_expect_tx(b_kv_full, 2 * C::TILE);
       for (int r = 0; r < C::N_REG; ++r) {
-        tma_load_3d(sK + r * C::REG, &tm_k, b_kv_full, r * 64, k0, bh);
-        tma_load_3d(sV + r * C::REG, &tm_v, b_kv_full, r * 64, k0, bh);
+        tma_load_4d(sK + r * C::REG, &tm_k, b_kv_full, r * 64, sp.k0 + k0, h_kv, sp.bc);
+        tma_load_4d(sV + r * C::REG, &tm_v, b_kv_full, r * 64, sp.k0 + k0, h_kv, sp.bc);
       }
       for (int it = 0; it < n_iter; ++it) {
         const int s = it & 1;
@@ -291,15 +379,17 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // Q_i with its lse2 and D rows; the stage is released after dK_i
         if (round > 0 && !mbar_wait(b_q_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
         mbar_expect_tx(b_q_full(s), C::TILE + C::VEC_BYTES);
-        for (int r = 0; r < C::N_REG; ++r) tma_load_3d(sQ(s) + r * C::REG, &tm_q, b_q_full(s), r * 64, q0, hq);
-        const size_t voff = static_cast<size_t>(hq) * args.Np + q0;
+        for (int r = 0; r < C::N_REG; ++r)
+          tma_load_4d(sQ(s) + r * C::REG, &tm_q, b_q_full(s), r * 64, sp.q0 + q0, hq, sp.bc);
+        const size_t voff = (static_cast<size_t>(b) * args.L.H + hq) * args.Np + q0;
         bulk_load(sVec(s), args.lse2 + voff, C::BM * 4, b_q_full(s));
         bulk_load(sVec(s) + C::BM * 4, args.dvec + voff, C::BM * 4, b_q_full(s));
         q_last[s] = it;
         // dO_i; the stage is released after dV_i
         if (round > 0 && !mbar_wait(b_do_empty(s), (round - 1) & 1, ctl)) { ok = false; break; }
         mbar_expect_tx(b_do_full(s), C::TILE);
-        for (int r = 0; r < C::N_REG; ++r) tma_load_3d(sDO(s) + r * C::REG, &tm_do, b_do_full(s), r * 64, q0, hq);
+        for (int r = 0; r < C::N_REG; ++r)
+          tma_load_4d(sDO(s) + r * C::REG, &tm_do, b_do_full(s), r * 64, sp.q0 + q0, hq, sp.bc);
         do_last[s] = it;
       }
       if (!ok) {       // let the loads in flight land before the CTA exits
@@ -408,7 +498,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t tX = tmem + lane_off + C::T_X + 64 * ch;
     const uint32_t tP = tmem + lane_off + C::T_Y + 32 * ch;     // this thread's 64 P values, packed
     const float c2 = args.scale_log2;
-    const bool key_ok = key < args.N;
+    const bool key_ok = key < sp.nk;
     // this thread's half row of the dS tile: region ch, row rloc; 16-byte
     // chunk j of the row sits at chunk j ^ (row & 7) (128-byte swizzle)
     uint8_t* prow = smem + C::OFF_PS + ch * C::REG + rloc * 128;
@@ -458,8 +548,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           }
         }
       }
-      // keys past the sequence end, and (causal) queries before this key, get P = 0
-      const int cut = !key_ok ? C::BM : (args.causal ? key - q0 : 0);   // columns c < cut are masked
+      // keys past the sequence end, and (causal) queries that do not see this key, get P = 0
+      const int cut = !key_ok ? C::BM : (args.causal ? key - off - q0 : 0);   // columns c < cut are masked
       if (cut > 64 * ch) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
@@ -506,11 +596,11 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // ---- epilogue: this thread's half of the dV, dK rows (D / 2 columns) -> global
     if (ok && mbar_wait_warp(b_dkv_done, 0, ctl)) {
       tc_fence_after();
-      const size_t grow = (static_cast<size_t>(bh) * args.N + key) * D + (D / 2) * ch;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t tsrc = tmem + lane_off + (which ? C::T_DK : C::T_DV) + (D / 2) * ch;
-        __nv_bfloat16* dst = (which ? args.dk : args.dv) + grow;
+        __nv_bfloat16* dst = which ? args.dk + row_offset(args.sdk, sp.bc, h_kv, sp.k0 + key) + (D / 2) * ch
+                                   : args.dv + row_offset(args.sdv, sp.bc, h_kv, sp.k0 + key) + (D / 2) * ch;
         const float mul = which ? args.scale : 1.0f;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
@@ -542,8 +632,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (!mbar_wait_warp(b_dq_full, static_cast<uint32_t>(it) & 1, ctl)) break;
       tc_fence_after();
       const int q0 = q_row0(it);
-      float* acc = args.dq_acc + static_cast<size_t>(q_head(it)) * args.N * D + dl;
-      const int nq = min(C::BM, args.N - q0);
+      float* acc = args.dq_acc + row_index<PACKED>(args.L, sp, q_head(it), q0) * D + dl;
+      const int nq = min(C::BM, sp.nq - q0);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {      // two 64-column halves (register budget), each released once loaded
         uint32_t r[64];
@@ -554,7 +644,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r + 32));
         tc_fence_before();
         mbar_arrive(h == 0 ? b_ylo_free : b_yhi_free);
-        float* a_row = acc + static_cast<size_t>(q0 + 64 * h) * D;
+        float* a_row = acc + static_cast<size_t>(64 * h) * D;
         // valid rows in this half (may be <= 0); none for the lanes past the head dim (D = 64)
         const int nh = dl < D ? nq - 64 * h : 0;
         if (nh >= 64) {

@@ -26,7 +26,8 @@ struct DevState {
   bool ready = false;
   uint32_t* status = nullptr;
   int sms = 0;
-  bool fwd_attr64 = false, fwd_attr128 = false, bwd_attr64 = false, bwd_attr128 = false, dec_attr = false;
+  bool fwd_attr[2][2] = {}, bwd_attr[2][2] = {};   // [d == 128][packed]: attributes set, registers checked
+  bool dec_attr = false;
 };
 DevState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -73,6 +74,105 @@ fa_status check_sizes(int B, int H, int N, int d, float scale) {
   if (numel >= (1LL << 31)) return FA_ERR_INVALID;
   return FA_OK;
 }
+
+// 4-D bf16 tensor map over [batch][head][row][d] with element strides st:
+// box {64 columns, 128 rows, 1 head, 1 batch entry}, 128-byte swizzle (the
+// layout the UMMA descriptors in the kernels expect).  Extents of 1 get a
+// harmless dense stride (the copy never steps along them); an extent of 0
+// rows is mapped as 1 row that no copy reads.
+bool make_map4(CUtensorMap* m, const void* base, int d, int rows, int heads, int batches, const fa_strides& st) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  if (rows < 1) rows = 1;
+  const cuuint64_t dense = static_cast<cuuint64_t>(d) * 2;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(batches)};
+  cuuint64_t strides[3] = {rows > 1 ? static_cast<cuuint64_t>(st.row) * 2 : dense,
+                           heads > 1 ? static_cast<cuuint64_t>(st.head) * 2 : dense,
+                           batches > 1 ? static_cast<cuuint64_t>(st.batch) * 2 : dense};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+fa_strides dense_strides(int H, int N, int d) {
+  fa_strides st;
+  st.row = d;
+  st.head = static_cast<int64_t>(N) * d;
+  st.batch = static_cast<int64_t>(H) * N * d;
+  return st;
+}
+
+// The layout of dense [B, H, N, d] tensors (H_kv heads for k, v, dk, dv).
+fa_layout dense_layout(int B, int H, int H_kv, int N, int d) {
+  fa_layout L = {};
+  L.B = B;
+  L.H = H;
+  L.H_kv = H_kv;
+  L.d = d;
+  L.Nq = L.Nk = N;
+  L.cu_seqlens_q = L.cu_seqlens_k = nullptr;
+  L.total_q = L.total_k = 0;
+  L.q = L.o = L.dout = L.dq = dense_strides(H, N, d);
+  L.k = L.v = L.dk = L.dv = dense_strides(H_kv, N, d);
+  return L;
+}
+
+bool packed(const fa_layout& L) { return L.cu_seqlens_q != nullptr; }
+int q_rows(const fa_layout& L) { return packed(L) ? L.total_q : L.Nq; }   // row extent of q-like tensors
+int k_rows(const fa_layout& L) { return packed(L) ? L.total_k : L.Nk; }
+int batches(const fa_layout& L) { return packed(L) ? 1 : L.B; }
+
+// Strides usable by TMA and by 16-byte row stores: positive multiples of 8
+// elements (16 bytes of bf16) below 2^38 (a tensor map stride is under 2^40 B).
+bool strides_ok(const fa_strides& st, int rows, int heads, int batches) {
+  auto ok = [](int64_t x, int extent) { return extent <= 1 || (x > 0 && x % 8 == 0 && x < (int64_t(1) << 38)); };
+  return ok(st.row, rows) && ok(st.head, heads) && ok(st.batch, batches);
+}
+
+// Sizes and strides of a layout (the pointers are checked by the caller).
+fa_status check_layout(const fa_layout& L, bool bwd) {
+  if (L.B < 1 || L.H < 1 || L.H_kv < 1 || L.H % L.H_kv != 0) return FA_ERR_INVALID;
+  if (L.Nq < 0 || L.Nk < 0 || L.Nq > (1 << 24) || L.Nk > (1 << 24)) return FA_ERR_INVALID;
+  if ((L.cu_seqlens_q == nullptr) != (L.cu_seqlens_k == nullptr)) return FA_ERR_INVALID;
+  if (packed(L)) {
+    if (L.total_q < 0 || L.total_k < 0 || L.B > (1 << 24)) return FA_ERR_INVALID;
+    if (reinterpret_cast<uintptr_t>(L.cu_seqlens_q) % 4 || reinterpret_cast<uintptr_t>(L.cu_seqlens_k) % 4)
+      return FA_ERR_ALIGN;
+  }
+  if (L.d != 64 && L.d != 128) return FA_ERR_UNSUPPORTED;
+  // every row index the kernels form stays below 2^31
+  const long long qr = static_cast<long long>(batches(L)) * L.H * (packed(L) ? L.total_q : L.Nq);
+  const long long pr = static_cast<long long>(L.B) * L.H * ((static_cast<long long>(L.Nq) + 127) / 128 * 128);
+  if (qr >= (1LL << 31) || pr >= (1LL << 31)) return FA_ERR_INVALID;
+  const int bq = batches(L), nq = q_rows(L), nk = k_rows(L);
+  if (!strides_ok(L.q, nq, L.H, bq) || !strides_ok(L.o, nq, L.H, bq) || !strides_ok(L.k, nk, L.H_kv, bq) ||
+      !strides_ok(L.v, nk, L.H_kv, bq))
+    return FA_ERR_ALIGN;
+  if (bwd && (!strides_ok(L.dout, nq, L.H, bq) || !strides_ok(L.dq, nq, L.H, bq) ||
+              !strides_ok(L.dk, nk, L.H_kv, bq) || !strides_ok(L.dv, nk, L.H_kv, bq)))
+    return FA_ERR_ALIGN;
+  return FA_OK;
+}
+
+SeqLayout seq_layout(const fa_layout& L) {
+  SeqLayout s;
+  s.cu_q = L.cu_seqlens_q;
+  s.cu_k = L.cu_seqlens_k;
+  s.B = L.B;
+  s.H = L.H;
+  s.H_kv = L.H_kv;
+  s.Nq = L.Nq;
+  s.Nk = L.Nk;
+  s.total_q = L.total_q;
+  s.total_k = L.total_k;
+  return s;
+}
+
+Strides kstrides(const fa_strides& st) { return Strides{st.batch, st.head, st.row}; }
 
 // 3-D bf16 tensor map over [BH][N][d]: box {64 columns, box_rows rows, 1 head},
 // 128-byte swizzle (the layout the UMMA descriptors in the kernels expect).
@@ -127,38 +227,38 @@ bool launch_regs_are(const void* fn, int regs) {
 
 template <int D>
 fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, void* o, float* lse,
-                     int B, int H, int H_kv, int N, float scale, int causal, int o_f32, cudaStream_t stream) {
-  const int BH = B * H;
+                     const fa_layout& L, float scale, int causal, int o_f32, cudaStream_t stream) {
   using C = FwdCfg<D>;
-  bool& attr = (D == 64) ? ds->fwd_attr64 : ds->fwd_attr128;
+  const bool pk = packed(L);
+  auto kern = pk ? fa_fwd_kernel<D, true> : fa_fwd_kernel<D, false>;
+  bool& attr = ds->fwd_attr[D == 128][pk];
   if (!attr) {
-    if (!launch_regs_are(reinterpret_cast<const void*>(fa_fwd_kernel<D>), C::LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(fa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
+    if (!launch_regs_are(reinterpret_cast<const void*>(kern), C::LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return FA_ERR_CUDA;
     attr = true;
   }
+  if (L.Nq == 0 || (packed(L) && L.total_q == 0)) return FA_OK;   // no query row: nothing to write
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, D, N, BH, 128) || !make_map(&tk, k, D, N, B * H_kv, 128) ||
-      !make_map(&tv, v, D, N, B * H_kv, 128))
+  const int bq = batches(L);
+  if (!make_map4(&tq, q, D, q_rows(L), L.H, bq, L.q) || !make_map4(&tk, k, D, k_rows(L), L.H_kv, bq, L.k) ||
+      !make_map4(&tv, v, D, k_rows(L), L.H_kv, bq, L.v))
     return FA_ERR_CUDA;
   FwdArgs a;
   a.o = o;
   a.lse = lse;
   a.status = ds->status;
-  a.N = N;
-  a.bh = BH;
-  a.heads = H;
-  a.group = H / H_kv;
-  a.n_qt = (N + 255) / 256;
-  a.n_kv_all = (N + 127) / 128;
-  a.num_tiles = BH * a.n_qt;
+  a.L = seq_layout(L);
+  a.so = kstrides(L.o);
+  a.group = L.H / L.H_kv;
+  a.n_qt = (L.Nq + 255) / 256;
+  a.num_tiles = L.B * L.H * a.n_qt;
   a.causal = causal ? 1 : 0;
   a.o_f32 = o_f32;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.wait_limit_ns = kWaitLimitNs;
   const int grid = a.num_tiles < ds->sms ? a.num_tiles : ds->sms;
-  fa_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -195,8 +295,23 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     vv = w + 2 * part;
   }
   const int of32 = dtype == FA_F32 ? 1 : 0;
-  return d == 64 ? launch_fwd<64>(ds, qq, kk, vv, o, lse, B, H, H_kv, N, scale, causal, of32, stream)
-                 : launch_fwd<128>(ds, qq, kk, vv, o, lse, B, H, H_kv, N, scale, causal, of32, stream);
+  const fa_layout L = dense_layout(B, H, H_kv, N, d);
+  return d == 64 ? launch_fwd<64>(ds, qq, kk, vv, o, lse, L, scale, causal, of32, stream)
+                 : launch_fwd<128>(ds, qq, kk, vv, o, lse, L, scale, causal, of32, stream);
+}
+
+fa_status fwd_general_impl(const void* q, const void* k, const void* v, void* o, float* lse, const fa_layout* Lp,
+                           float scale, int causal, cudaStream_t stream) {
+  if (Lp == nullptr) return FA_ERR_INVALID;
+  const fa_layout& L = *Lp;
+  fa_status st = check_layout(L, false);
+  if (st != FA_OK) return st;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
+  DevState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  return L.d == 64 ? launch_fwd<64>(ds, q, k, v, o, lse, L, scale, causal, 0, stream)
+                   : launch_fwd<128>(ds, q, k, v, o, lse, L, scale, causal, 0, stream);
 }
 
 }  // namespace
@@ -230,11 +345,29 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
                   static_cast<cudaStream_t>(stream));
 }
 
+fa_status fa_fwd_general(const void* q, const void* k, const void* v, void* o, float* lse, const fa_layout* layout,
+                         float scale, int causal, fa_stream_t stream) {
+  return fwd_general_impl(q, k, v, o, lse, layout, scale, causal, static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+// fp32 dQ accumulator (one row per query row and head), then lse * log2(e) and
+// D for rows padded to a multiple of 128 per (sequence, head).
+size_t bwd_ws_bytes(const fa_layout& L) {
+  const size_t acc_rows = packed(L) ? static_cast<size_t>(L.H) * L.total_q : static_cast<size_t>(L.B) * L.H * L.Nq;
+  const size_t np = (static_cast<size_t>(L.Nq) + 127) / 128 * 128;
+  return round256(acc_rows * L.d * 4) + 2 * round256(static_cast<size_t>(L.B) * L.H * np * 4);
+}
+}  // namespace
+
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
-  const size_t bh = static_cast<size_t>(B) * H;
-  const size_t np = (static_cast<size_t>(N) + 127) / 128 * 128;
-  return round256(bh * N * d * 4) + 2 * round256(bh * np * 4);
+  return bwd_ws_bytes(dense_layout(B, H, H, N, d));
+}
+
+size_t fa_bwd_general_workspace_size(const fa_layout* layout) {
+  if (layout == nullptr || check_layout(*layout, true) != FA_OK) return 0;
+  return bwd_ws_bytes(*layout);
 }
 
 }  // extern "C"
@@ -244,47 +377,61 @@ namespace {
 
 enum BwdPhase : int { PH_PREPARE = 1, PH_MAIN = 2, PH_FINISH = 4, PH_ALL = 7 };
 
-// First use of the backward main kernel for head dim D on a device.
-template <int D>
+// First use of a backward main kernel on a device.
+template <int D, bool PACKED>
 fa_status prepare_bwd_kernel() {
   using C = BwdCfg<D>;
-  if (!launch_regs_are(reinterpret_cast<const void*>(fa_bwd_kernel<D>), C::LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(fa_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+  if (!launch_regs_are(reinterpret_cast<const void*>(fa_bwd_kernel<D, PACKED>), C::LAUNCH_REGS))
+    return FA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(fa_bwd_kernel<D, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;
 }
 
+template <int D>
+void launch_bwd_main(bool pk, unsigned grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  if (pk)
+    fa_bwd_kernel<D, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  else
+    fa_bwd_kernel<D, false><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+}
+
 // Validates, fills the kernel arguments, and launches the requested phases.
 fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, const void* o, const float* lse,
-                   const void* dout, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
-                   float scale, int causal, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  fa_status st = check_sizes(B, H, N, d, scale);
+                   const void* dout, void* dq, void* dk, void* dv, const fa_layout& L, float scale, int causal,
+                   void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  fa_status st = check_layout(L, true);
   if (st != FA_OK) return st;
-  if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID;
+  const int d = L.d;
   if ((phases & PH_PREPARE) && (!aligned16(o) || !aligned16(lse) || !aligned16(dout))) return FA_ERR_ALIGN;
   if ((phases & PH_MAIN) && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
                              !aligned16(dk) || !aligned16(dv)))
     return FA_ERR_ALIGN;
   if ((phases & PH_FINISH) && !aligned16(dq)) return FA_ERR_ALIGN;
-  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  const size_t need = bwd_ws_bytes(L);
   if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return FA_ERR_WORKSPACE;
   DevState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
-  if ((phases & PH_MAIN) && !(d == 64 ? ds->bwd_attr64 : ds->bwd_attr128)) {
-    st = d == 64 ? prepare_bwd_kernel<64>() : prepare_bwd_kernel<128>();
+  const bool pk = packed(L);
+  if ((phases & PH_MAIN) && !ds->bwd_attr[d == 128][pk]) {
+    st = d == 64 ? (pk ? prepare_bwd_kernel<64, true>() : prepare_bwd_kernel<64, false>())
+                 : (pk ? prepare_bwd_kernel<128, true>() : prepare_bwd_kernel<128, false>());
     if (st != FA_OK) return st;
-    (d == 64 ? ds->bwd_attr64 : ds->bwd_attr128) = true;
+    ds->bwd_attr[d == 128][pk] = true;
   }
-  const int BH = B * H;
   BwdArgs a;
-  const size_t np = (static_cast<size_t>(N) + 127) / 128 * 128;
+  const size_t np = (static_cast<size_t>(L.Nq) + 127) / 128 * 128;
+  a.acc_rows = packed(L) ? static_cast<long long>(L.H) * L.total_q : static_cast<long long>(L.B) * L.H * L.Nq;
   uint8_t* w = static_cast<uint8_t*>(workspace);
   a.dq_acc = reinterpret_cast<float*>(w);
-  a.lse2 = reinterpret_cast<float*>(w + round256(static_cast<size_t>(BH) * N * d * 4));
-  a.dvec = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.lse2) + round256(BH * np * 4));
+  a.lse2 = reinterpret_cast<float*>(w + round256(static_cast<size_t>(a.acc_rows) * d * 4));
+  a.dvec = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.lse2) +
+                                    round256(static_cast<size_t>(L.B) * L.H * np * 4));
   a.o = static_cast<const __nv_bfloat16*>(o);
   a.dout = static_cast<const __nv_bfloat16*>(dout);
   a.lse = lse;
@@ -292,16 +439,22 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
   a.status = ds->status;
-  a.N = N;
+  a.L = seq_layout(L);
+  a.so = kstrides(L.o);
+  a.sdo = kstrides(L.dout);
+  a.sdq = kstrides(L.dq);
+  a.sdk = kstrides(L.dk);
+  a.sdv = kstrides(L.dv);
+  const fa_strides dd = dense_strides(L.H, L.Nq, d);
+  a.dq_dense = !packed(L) && (L.Nq <= 1 || L.dq.row == dd.row) && (L.H <= 1 || L.dq.head == dd.head) &&
+               (L.B <= 1 || L.dq.batch == dd.batch);
   a.Np = static_cast<int>(np);
-  a.bh = BH;
-  a.bh_kv = B * H_kv;
-  a.heads = H;
-  a.group = H / H_kv;
-  a.n_kb = (N + 127) / 128;
-  a.n_qb = (N + 127) / 128;
+  a.bh_kv = L.B * L.H_kv;
+  a.group = L.H / L.H_kv;
+  a.n_kb = (L.Nk + 127) / 128;
   // enough key/value heads per scheduling group to fill the GPU about twice over with key blocks
-  const int want = (2 * ds->sms + a.n_kb - 1) / a.n_kb;
+  const int nkb = a.n_kb < 1 ? 1 : a.n_kb;
+  const int want = (2 * ds->sms + nkb - 1) / nkb;
   a.heads_per_group = want < 1 ? 1 : (want > a.bh_kv ? a.bh_kv : want);
   a.causal = causal ? 1 : 0;
   a.scale = scale;
@@ -313,18 +466,20 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
     else
       fa_bwd_pre_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
   }
-  if (phases & PH_MAIN) {
+  if ((phases & PH_MAIN) && a.n_kb > 0 && !(packed(L) && L.total_k == 0)) {
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_map(&tq, q, d, N, BH, 128) || !make_map(&tk, k, d, N, a.bh_kv, 128) ||
-        !make_map(&tv, v, d, N, a.bh_kv, 128) || !make_map(&tdo, dout, d, N, BH, 128))
+    const int bq = batches(L);
+    if (!make_map4(&tq, q, d, q_rows(L), L.H, bq, L.q) || !make_map4(&tk, k, d, k_rows(L), L.H_kv, bq, L.k) ||
+        !make_map4(&tv, v, d, k_rows(L), L.H_kv, bq, L.v) || !make_map4(&tdo, dout, d, q_rows(L), L.H, bq, L.dout))
       return FA_ERR_CUDA;
+    const long long grid = static_cast<long long>(a.n_kb) * a.bh_kv;
+    if (grid >= (1LL << 31)) return FA_ERR_INVALID;
     if (d == 64)
-      fa_bwd_kernel<64><<<a.n_kb * a.bh_kv, BwdCfg<64>::THREADS, BwdCfg<64>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+      launch_bwd_main<64>(pk, static_cast<unsigned>(grid), tq, tk, tv, tdo, a, stream);
     else
-      fa_bwd_kernel<128><<<a.n_kb * a.bh_kv, BwdCfg<128>::THREADS, BwdCfg<128>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo,
-                                                                                                       a);
+      launch_bwd_main<128>(pk, static_cast<unsigned>(grid), tq, tk, tv, tdo, a, stream);
   }
-  if (phases & PH_FINISH) {
+  if ((phases & PH_FINISH) && a.acc_rows > 0) {
     if (d == 64)
       fa_bwd_dq_kernel<64><<<ds->sms * 8, 256, 0, stream>>>(a);
     else
@@ -341,34 +496,47 @@ extern "C" {
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                  void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  return bwd_impl(PH_ALL, q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, scale, causal, workspace,
+  if (check_sizes(B, H, N, d, scale) != FA_OK) return FA_ERR_INVALID;
+  return bwd_impl(PH_ALL, q, k, v, o, lse, dout, dq, dk, dv, dense_layout(B, H, H, N, d), scale, causal, workspace,
                   workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dout, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
                      float scale, int causal, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  return bwd_impl(PH_ALL, q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, scale, causal, workspace,
-                  workspace_bytes, static_cast<cudaStream_t>(stream));
+  if (check_sizes(B, H, N, d, scale) != FA_OK || H_kv < 1) return FA_ERR_INVALID;
+  return bwd_impl(PH_ALL, q, k, v, o, lse, dout, dq, dk, dv, dense_layout(B, H, H_kv, N, d), scale, causal,
+                  workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd_general(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, const fa_layout* layout, float scale,
+                         int causal, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  if (layout == nullptr) return FA_ERR_INVALID;
+  return bwd_impl(PH_ALL, q, k, v, o, lse, dout, dq, dk, dv, *layout, scale, causal, workspace, workspace_bytes,
+                  static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_bwd_prepare(const void* o, const float* lse, const void* dout, int B, int H, int N, int d,
                          void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  return bwd_impl(PH_PREPARE, nullptr, nullptr, nullptr, o, lse, dout, nullptr, nullptr, nullptr, B, H, H, N, d,
-                  1.0f, 0, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+  if (check_sizes(B, H, N, d, 1.0f) != FA_OK) return FA_ERR_INVALID;
+  return bwd_impl(PH_PREPARE, nullptr, nullptr, nullptr, o, lse, dout, nullptr, nullptr, nullptr,
+                  dense_layout(B, H, H, N, d), 1.0f, 0, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B,
                       int H, int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
                       fa_stream_t stream) {
-  return bwd_impl(PH_MAIN, q, k, v, nullptr, nullptr, dout, nullptr, dk, dv, B, H, H, N, d, scale, causal,
-                  workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+  if (check_sizes(B, H, N, d, scale) != FA_OK) return FA_ERR_INVALID;
+  return bwd_impl(PH_MAIN, q, k, v, nullptr, nullptr, dout, nullptr, dk, dv, dense_layout(B, H, H, N, d), scale,
+                  causal, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_bwd_finish(void* dq, int B, int H, int N, int d, float scale, void* workspace,
                         size_t workspace_bytes, fa_stream_t stream) {
-  return bwd_impl(PH_FINISH, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dq, nullptr, nullptr, B, H,
-                  H, N, d, scale, 0, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+  if (check_sizes(B, H, N, d, scale) != FA_OK) return FA_ERR_INVALID;
+  return bwd_impl(PH_FINISH, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dq, nullptr, nullptr,
+                  dense_layout(B, H, H, N, d), scale, 0, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 // ---- backward with built-in scratch (no allocation) ----
@@ -415,7 +583,8 @@ fa_status fa_get_device_status(fa_stream_t stream) {
   if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
   if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
   if (v & DEV_TIMEOUT) return FA_ERR_TIMEOUT;
-  return (v & DEV_SMEM) ? FA_ERR_CUDA : FA_OK;
+  if (v & DEV_SMEM) return FA_ERR_CUDA;
+  return (v & DEV_ARGS) ? FA_ERR_INVALID : FA_OK;
 }
 
 fa_status fa_selftest_wait_timeout(uint64_t timeout_ns, fa_stream_t stream) {

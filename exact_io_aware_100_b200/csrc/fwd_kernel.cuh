@@ -11,7 +11,10 @@
 //
 // B200 design (not the pages' A100 / H100 partitioning):
 //  * persistent CTAs, one per SM, walk work tiles of 256 query rows of one
-//    (batch, head); causal tiles are visited longest first;
+//    (sequence, head); causal tiles are visited longest first;
+//  * any query and key lengths, fixed per batch entry or packed variable-length
+//    sequences, and any row / head / batch strides (layout.cuh); TMA reads the
+//    tiles through 4-D tensor maps [d][row][head][batch];
 //  * warp roles: warps 0-3 and 4-7 are two softmax warpgroups, each owning one
 //    128-row half of the tile (thread t owns TMEM lane / query row t); warp 8
 //    issues the tcgen05 MMAs from one thread; warp 9 issues TMA loads from one
@@ -29,21 +32,20 @@
 //    drains its own in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
 
+#include "layout.cuh"
 #include "ptx.cuh"
 
 namespace fa {
 
 struct FwdArgs {
-  void* o;              // [BH, N, D] bf16 or f32
-  float* lse;           // [BH, N] natural-log logsumexp
+  void* o;              // bf16 or f32, strides so
+  float* lse;           // natural-log logsumexp, indexed by row_index
   uint32_t* status;     // device status word
-  int N;
-  int bh;               // B * H (query heads)
-  int heads;            // H
+  SeqLayout L;
+  Strides so;           // element strides of o
   int group;            // query heads per key/value head (1: multi-head; H: multi-query)
-  int n_qt;             // ceil(N / 256)
-  int n_kv_all;         // ceil(N / 128)
-  int num_tiles;        // bh * n_qt
+  int n_qt;             // ceil(L.Nq / 256)
+  int num_tiles;        // B * H * n_qt
   int causal;
   int o_f32;
   float scale_log2;     // scale * log2(e)
@@ -79,29 +81,35 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
 };
 
-__device__ __forceinline__ void fwd_decode_tile(const FwdArgs& a, int t, int& bh, int& qt) {
+// Work tile t -> (sequence b, query head h, tile qt of 256 query rows).  Query
+// head h reads key/value head h / group (sets of consecutive query heads share
+// one: grouped-query attention; group = 1 is multi-head).
+__device__ __forceinline__ void fwd_decode_tile(const FwdArgs& a, int t, int& b, int& h, int& qt) {
+  const int bh_all = a.L.B * a.L.H;
+  int bh;
   if (a.causal) {            // longest work first
-    qt = a.n_qt - 1 - t / a.bh;
-    bh = t % a.bh;
+    qt = a.n_qt - 1 - t / bh_all;
+    bh = t % bh_all;
   } else {                   // neighbouring CTAs share a head's K / V in L2
     bh = t / a.n_qt;
     qt = t % a.n_qt;
   }
+  b = bh / a.L.H;
+  h = bh - b * a.L.H;
 }
 
-// Key/value head of query head bh: sets of `group` consecutive query heads of a
-// batch entry share one (grouped-query attention; group = 1 is multi-head).
-__device__ __forceinline__ int fwd_kv_head(const FwdArgs& a, int bh) {
-  return (bh / a.heads) * (a.heads / a.group) + (bh % a.heads) / a.group;
+// Key blocks (128 keys) tile qt of sequence s reads; 0 when the tile holds no
+// query row or none of its rows sees a key (then its rows are written as empty).
+__device__ __forceinline__ int fwd_num_kv(const FwdArgs& a, const SeqSpan& s, int qt) {
+  if (qt * 256 >= s.nq) return 0;
+  const int n_all = (s.nk + 127) / 128;
+  if (!a.causal) return n_all;
+  const int last_row = min(qt * 256 + 255, s.nq - 1);
+  const int vis = last_row + (s.nk - s.nq) + 1;       // keys < vis are visible to the last row
+  return vis <= 0 ? 0 : min((vis + 127) / 128, n_all);
 }
 
-__device__ __forceinline__ int fwd_num_kv(const FwdArgs& a, int qt) {
-  if (!a.causal) return a.n_kv_all;
-  const int last_row = min(qt * 256 + 255, a.N - 1);
-  return last_row / 128 + 1;
-}
-
-template <int D>
+template <int D, bool PACKED>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
@@ -163,16 +171,19 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       bool ok = true, q_pending = false;
       uint32_t q_parity = 0;
       uint32_t issued = 0, last_parity = 0;      // per-stage bit masks
-      for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x, ++tile_cnt) {
-        int bh, qt;
-        fwd_decode_tile(args, t, bh, qt);
-        const int nkv = fwd_num_kv(args, qt);
-        const int bh_kv = fwd_kv_head(args, bh);
+      for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
+        int b, h, qt;
+        fwd_decode_tile(args, t, b, h, qt);
+        const SeqSpan sp = seq_span<PACKED>(args.L, b, args.status);
+        const int nkv = fwd_num_kv(args, sp, qt);
+        if (nkv == 0) continue;                        // nothing to load for this tile
+        const int h_kv = h / args.group;
         if (tile_cnt > 0 && !mbar_wait(b_q_empty, (tile_cnt - 1) & 1, ctl)) { ok = false; break; }
         mbar_expect_tx(b_q_full, 2 * C::Q_HALF);
-        for (int h = 0; h < 2; ++h)
+        for (int hf = 0; hf < 2; ++hf)
           for (int r = 0; r < C::N_REG; ++r)
-            tma_load_3d(sQ + h * C::Q_HALF + r * C::REGION, &tm_q, b_q_full, r * 64, qt * 256 + h * 128, bh);
+            tma_load_4d(sQ + hf * C::Q_HALF + r * C::REGION, &tm_q, b_q_full, r * 64, sp.q0 + qt * 256 + hf * 128,
+                        h, sp.bc);
         q_pending = true;
         q_parity = tile_cnt & 1;
         for (int j = 0; j < nkv && ok; ++j) {
@@ -183,11 +194,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_expect_tx(b_kv_full(s), C::KV_BYTES);
             const CUtensorMap* map = kind ? &tm_v : &tm_k;
             for (int r = 0; r < C::N_REG; ++r)
-              tma_load_3d(sKV + s * C::KV_BYTES + r * C::REGION, map, b_kv_full(s), r * 64, j * 128, bh_kv);
+              tma_load_4d(sKV + s * C::KV_BYTES + r * C::REGION, map, b_kv_full(s), r * 64, sp.k0 + j * 128, h_kv,
+                          sp.bc);
             issued |= 1u << s;
             last_parity = (last_parity & ~(1u << s)) | ((round & 1u) << s);
           }
         }
+        ++tile_cnt;
       }
       if (!ok) {   // drain our own copies still in flight before the CTA exits
         for (int s = 0; s < C::STAGES; ++s)
@@ -219,10 +232,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int kk = 0; kk < C::BN / 16; ++kk)
           umma_ts(d_tmem, p_tmem + kk * 8, dv + ((kk * 2048) >> 4), C::IDESC_PV, acc || (kk > 0));
       };
-      for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x, ++tile_cnt) {
-        int bh, qt;
-        fwd_decode_tile(args, t, bh, qt);
-        const int nkv = fwd_num_kv(args, qt);
+      for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
+        int b, h, qt;
+        fwd_decode_tile(args, t, b, h, qt);
+        const int nkv = fwd_num_kv(args, seq_span<PACKED>(args.L, b, args.status), qt);
+        if (nkv == 0) continue;
         if (!mbar_wait(b_q_full, tile_cnt & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         int sv_prev = 0;
@@ -266,6 +280,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         issue_pv(tmem + C::T_O1, tmem + C::T_S1, sKV + sv_prev * C::KV_BYTES, nkv > 1);
         umma_commit(b_kv_empty(sv_prev));
         umma_commit(b_o_done);
+        ++tile_cnt;
       }
       // every MMA issued by this thread has completed before TMEM is freed
       umma_commit(b_drain);
@@ -284,14 +299,31 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const float c2 = args.scale_log2;
     uint32_t s_par = 0, tile_cnt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x, ++tile_cnt) {
-      int bh, qt;
-      fwd_decode_tile(args, t, bh, qt);
-      const int nkv = fwd_num_kv(args, qt);
-      const int row0 = qt * 256 + half * 128;
+    for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
+      int b, h, qt;
+      fwd_decode_tile(args, t, b, h, qt);
+      const SeqSpan sp = seq_span<PACKED>(args.L, b, args.status);
+      const int nkv = fwd_num_kv(args, sp, qt);
+      const int row0 = qt * 256 + half * 128;           // rows of the sequence
       const int row = row0 + rloc;
-      const int lim = args.causal ? min(row + 1, args.N) : args.N;         // keys < lim are visible
-      const int lim_min = args.causal ? min(row0 + 1, args.N) : args.N;    // smallest lim in the warpgroup
+      if (nkv == 0) {                                   // no key visible to any row: O = 0, lse = -inf
+        if (row < sp.nq) {
+          const long long o_off = row_offset(args.so, sp.bc, h, sp.q0 + row);
+          const long long l_idx = row_index<PACKED>(args.L, sp, h, row);
+          if (args.o_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.o) + o_off);
+            for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.o) + o_off);
+            for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+          }
+          args.lse[l_idx] = -INFINITY;
+        }
+        continue;
+      }
+      const int off = sp.nk - sp.nq;                    // bottom-right causal alignment
+      const int lim = args.causal ? min(row + off + 1, sp.nk) : sp.nk;        // keys < lim are visible
+      const int lim_min = args.causal ? min(row0 + off + 1, sp.nk) : sp.nk;   // smallest lim in the warpgroup
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < nkv; ++j) {
         if (!mbar_wait_warp(b_s_full, s_par, ctl)) { ok = false; break; }
@@ -327,18 +359,21 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mx1 = fmax3(mx1, s[126], s[127]);
         const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
         const float m_new = fmaxf(m_ref, mx);
-        const bool need = (m_new - m_ref) * c2 > 8.0f;
+        const bool need = (m_new - m_ref) * c2 > 8.0f;          // false while the row has seen no key
         const bool rescale = __any_sync(0xffffffffu, need);   // warp-uniform decision
         float alpha = 1.0f;
         if (rescale) {
-          alpha = ex2_approx((m_ref - m_new) * c2);              // 0 on the first block
+          // 0 on a row's first visible key (m_ref = -inf); 1 while it has seen none
+          alpha = m_new == -INFINITY ? 1.0f : ex2_approx((m_ref - m_new) * c2);
           l *= alpha;
           m_ref = m_new;
         }
         // p = 2^(s c2 - m c2): three of every eight pairs on the FMA pipe, the rest
-        // on the special-function unit
+        // on the special-function unit.  A row that has seen no key yet has only
+        // masked scores here, and a finite reference keeps them at (about) zero.
         const float2 c2v = make_float2(c2, c2);
-        const float2 negm = make_float2(-m_ref * c2, -m_ref * c2);
+        const float m_use = m_ref == -INFINITY ? 0.0f : m_ref;
+        const float2 negm = make_float2(-m_use * c2, -m_use * c2);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         uint32_t pr[64];
 #pragma unroll
@@ -385,9 +420,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // ---- epilogue: O / l -> global, lse
       if (!mbar_wait_warp(b_o_done, tile_cnt & 1, ctl)) { ok = false; break; }
       tc_fence_after();
-      const float inv_l = 1.0f / l;
-      const bool valid = row < args.N;
-      const size_t grow = static_cast<size_t>(bh) * args.N + row;
+      // a row that saw no key (m_ref still -inf) is written as O = 0, lse = -inf
+      const bool seen = m_ref != -INFINITY;
+      const float inv_l = seen ? 1.0f / l : 0.0f;
+      const SeqSpan spe = seq_span<PACKED>(args.L, b, args.status);   // addresses formed after the loop
+      const bool valid = row < spe.nq;
+      const long long o_off = row_offset(args.so, spe.bc, h, spe.q0 + row);
+      const long long l_idx = row_index<PACKED>(args.L, spe, h, row);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -396,13 +435,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         reg_fence32(o);
         if (valid) {
           if (args.o_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.o) + grow * D + c * 32);
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.o) + o_off + c * 32);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
                                    __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.o) + grow * D + c * 32);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.o) + o_off + c * 32);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               uint4 w;
@@ -415,7 +454,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           }
         }
       }
-      if (valid) args.lse[grow] = (m_ref * c2 + __log2f(l)) * 0.69314718055994531f;
+      if (valid) args.lse[l_idx] = seen ? (m_ref * c2 + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      ++tile_cnt;
     }
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");   // warps 10-11: set-up and teardown only

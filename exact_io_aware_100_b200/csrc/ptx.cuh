@@ -20,6 +20,7 @@ enum : uint32_t {
   DEV_OK = 0u,
   DEV_TIMEOUT = 1u,      // a bounded mbarrier wait gave up
   DEV_SMEM = 2u,         // a kernel's shared-memory plan did not fit its allocation
+  DEV_ARGS = 4u,         // device-side arguments (sequence offsets) were inconsistent
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -112,6 +113,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 // Plain (untiled) bulk copy global -> shared; both addresses 16-byte aligned,

@@ -14,8 +14,8 @@
  * recomputation") and returns the exact gradients
  *     dV = P^T dO,  dS = P * (dO V^T - D),  D_i = sum_c dO_ic O_ic,
  *     dQ = scale dS K,  dK = scale dS^T Q.
- * Causal masking hides key j from query i when j > i (top-left aligned,
- * equal query and key lengths).
+ * Causal masking hides key j from query i when j > i (equal query and key
+ * lengths; the general-layout calls below align it bottom-right).
  *
  * Conventions shared by every call:
  *  - Layout: q, k, v, o, dO, dq, dk, dv are dense row-major [B, H, N, d] with d
@@ -140,6 +140,75 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
                      void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * General lengths and layouts.  The pages define attention for one square
+ * sequence; the integrations they point users to (deepfa.ir, "Flash
+ * Attention: بهینه‌سازی مکانیزم توجه در ترنسفورمرها", section on
+ * implementation and use: PyTorch, Transformers, vLLM) call it on tensors of
+ * other shapes, which these calls accept:
+ *  - any number of query rows Nq and key rows Nk (either may be 0);
+ *  - fixed lengths (every batch entry has Nq queries and Nk keys) or packed
+ *    variable lengths (sequence b is rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]
+ *    of the query tensors and cu_seqlens_k[b] .. cu_seqlens_k[b+1] of the
+ *    key / value tensors, as in a token-major [total, H, d] batch);
+ *  - any element strides for the batch, head and row axes (d contiguous), so
+ *    that [B, H, N, d], [B, N, H, d] and views of larger tensors need no copy;
+ *  - grouped heads as in fa_fwd_gqa.
+ * Causal masking is aligned bottom-right: query i of a sequence with nq
+ * queries and nk keys sees keys j <= nk - nq + i (the usual mask when
+ * nq == nk).  A query that sees no key (nq > nk under the causal mask, or
+ * nk == 0) gets o = 0 and lse = -inf, and contributes no gradient.
+ */
+typedef struct {
+  int64_t batch;   /* elements between batch entries (unused for packed sequences) */
+  int64_t head;    /* elements between heads                                    */
+  int64_t row;     /* elements between rows (tokens)                            */
+} fa_strides;
+
+typedef struct {
+  int B;                        /* batch entries (sequences)                                   */
+  int H, H_kv;                  /* query heads, key/value heads (H a multiple of H_kv)          */
+  int d;                        /* head dim: 64 or 128                                          */
+  int Nq, Nk;                   /* fixed lengths: rows per batch entry; packed: an upper bound
+                                   on every sequence's length (sets the grid)                   */
+  const int32_t* cu_seqlens_q;  /* packed: DEVICE array of B + 1 row offsets; NULL: fixed lengths */
+  const int32_t* cu_seqlens_k;  /* packed: likewise for keys and values; NULL with cu_seqlens_q  */
+  int total_q, total_k;         /* packed: rows of the query and key tensors (ignored otherwise) */
+  fa_strides q, k, v, o;        /* strides of the forward operands                               */
+  fa_strides dout, dq, dk, dv;  /* strides of the backward operands (the forward ignores them)   */
+} fa_layout;
+
+/*
+ * Forward with a general layout.  q, o: [batch][H][row][d] bf16 with strides
+ * layout->q, layout->o; k, v: [batch][H_kv][row][d] bf16.  lse (float, dense):
+ * [B, H, Nq] for fixed lengths, [H, total_q] for packed sequences.  Strides
+ * of axes longer than 1 must be positive multiples of 8 elements (16 bytes)
+ * (FA_ERR_ALIGN); every pointer non-null and 16-byte aligned.  Nq == 0 (or
+ * total_q == 0) launches nothing.  Packed offsets are read on the device: a
+ * sequence whose offsets are out of order, outside the tensors or longer
+ * than Nq / Nk is skipped (nothing written for it) and fa_get_device_status()
+ * then reports FA_ERR_INVALID.  Same ownership, stream and error rules as
+ * fa_fwd otherwise; `layout` is read during the call only.
+ */
+fa_status fa_fwd_general(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const fa_layout* layout, float scale, int causal, fa_stream_t stream);
+
+/*
+ * Backward with a general layout: the exact gradients of fa_fwd_general.
+ * Inputs q, k, v, o, dout (strides layout->q, k, v, o, dout) and lse from the
+ * forward (its layout); outputs dq, dk, dv (strides layout->dq, dk, dv),
+ * written, not accumulated; dk and dv of a shared head sum over its set.
+ * workspace: at least fa_bwd_general_workspace_size(layout) bytes, 256-byte
+ * aligned.  Same rules as fa_fwd_general and fa_bwd otherwise.
+ */
+fa_status fa_bwd_general(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, const fa_layout* layout,
+                         float scale, int causal, void* workspace, size_t workspace_bytes,
+                         fa_stream_t stream);
+
+/* Bytes of workspace fa_bwd_general needs (0 for a layout it rejects). */
+size_t fa_bwd_general_workspace_size(const fa_layout* layout);
+
+/*
  * Decoding: Lq queries that are the last Lq positions of a sequence of Nk keys
  * (a key/value cache), with the keys split across CTAs and the partial results
  * combined by the softmax merge of the unite.ai page "Flash Attention:
@@ -192,7 +261,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
  * current device.  Returns FA_ERR_TIMEOUT if any kernel since the last call
  * gave up a bounded wait, FA_ERR_CUDA if the synchronisation failed or a
  * kernel found its shared-memory allocation too small for its buffers (it then
- * did no work), else FA_OK.
+ * did no work), FA_ERR_INVALID if a kernel found inconsistent packed sequence
+ * offsets (it skipped those sequences), else FA_OK.
  */
 fa_status fa_get_device_status(fa_stream_t stream);
 

@@ -100,6 +100,83 @@ def test_decode_validation_without_device(lib):
     assert lib.fa_decode_workspace_size(2, 8, 3, 1, 1000, 128) == 0
 
 
+def test_layout_struct_matches_the_header(tmp_path):
+    """ctypes' fa_layout has the size and field offsets the C compiler gives include/fa.h's."""
+    import ctypes
+    import exact_io_aware_100_b200 as fa
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "fa.h"\n'
+        'int main(void) { printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(fa_layout), offsetof(fa_layout, cu_seqlens_q),'
+        ' offsetof(fa_layout, total_q), offsetof(fa_layout, q), offsetof(fa_layout, dv), sizeof(fa_strides));'
+        ' return 0; }\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    L = fa.FaLayout
+    assert got == [ctypes.sizeof(L), L.cu_seqlens_q.offset, L.total_q.offset, L.q.offset, L.dv.offset,
+                   ctypes.sizeof(fa.FaStrides)]
+
+
+def _dense_layout(fa, B, H, H_kv, Nq, Nk, d):
+    L = fa.FaLayout(B=B, H=H, H_kv=H_kv, d=d, Nq=Nq, Nk=Nk, cu_seqlens_q=None, cu_seqlens_k=None,
+                    total_q=0, total_k=0)
+    for n in ("q", "o", "dout", "dq"):
+        setattr(L, n, fa.FaStrides(H * Nq * d, Nq * d, d))
+    for n in ("k", "v", "dk", "dv"):
+        setattr(L, n, fa.FaStrides(H_kv * Nk * d, Nk * d, d))
+    return L
+
+
+def test_general_validation_without_device(lib):
+    import ctypes
+    import exact_io_aware_100_b200 as fa
+    P16 = 16
+    f, b = lib.fa_fwd_general, lib.fa_bwd_general
+    ref = ctypes.byref
+    assert f(P16, P16, P16, P16, P16, None, 0.1, 1, None) == 1                       # no layout
+    L = _dense_layout(fa, 2, 4, 2, 100, 300, 128)
+    assert f(P16, P16, P16, P16, P16 + 4, ref(L), 0.1, 1, None) == 3                 # misaligned lse
+    assert f(P16, P16, P16, P16, P16, ref(L), float("inf"), 1, None) == 1           # scale
+    bad = _dense_layout(fa, 2, 4, 2, 100, 300, 128)
+    bad.q = fa.FaStrides(4 * 100 * 128, 100 * 128, 132)                             # row stride not 16 B
+    assert f(P16, P16, P16, P16, P16, ref(bad), 0.1, 1, None) == 3
+    bad = _dense_layout(fa, 2, 4, 3, 100, 300, 128)                                   # uneven sets
+    assert f(P16, P16, P16, P16, P16, ref(bad), 0.1, 1, None) == 1
+    bad = _dense_layout(fa, 2, 4, 2, 100, 300, 96)                                    # d
+    assert f(P16, P16, P16, P16, P16, ref(bad), 0.1, 1, None) == 2
+    bad = _dense_layout(fa, 2, 4, 2, -1, 300, 128)                                    # negative length
+    assert f(P16, P16, P16, P16, P16, ref(bad), 0.1, 1, None) == 1
+    bad = _dense_layout(fa, 2, 4, 2, 100, 300, 128)
+    bad.cu_seqlens_q = 256                                                             # offsets for q only
+    assert f(P16, P16, P16, P16, P16, ref(bad), 0.1, 1, None) == 1
+    bad.cu_seqlens_k = 258                                                             # misaligned offsets
+    bad.total_q, bad.total_k = 100, 300
+    assert f(P16, P16, P16, P16, P16, ref(bad), 0.1, 1, None) == 3
+    args = [P16] * 9
+    assert b(*args, ref(L), 0.1, 1, None, 0, None) == 4                               # no workspace
+    need = lib.fa_bwd_general_workspace_size(ref(L))
+    assert b(*args, ref(L), 0.1, 1, 256, need - 1, None) == 4
+
+
+def test_general_workspace_sizes(lib):
+    import ctypes
+    import exact_io_aware_100_b200 as fa
+    L = _dense_layout(fa, 2, 4, 2, 100, 300, 128)
+    # fp32 dQ accumulator for B*H*Nq rows, then lse * log2(e) and D for rows padded to 128 per head
+    acc = 2 * 4 * 100 * 128 * 4
+    vec = (2 * 4 * 128 * 4 + 255) // 256 * 256
+    assert lib.fa_bwd_general_workspace_size(ctypes.byref(L)) == (acc + 255) // 256 * 256 + 2 * vec
+    # packed: H * total_q accumulator rows; the vectors are padded to the longest sequence
+    L.cu_seqlens_q, L.cu_seqlens_k, L.total_q, L.total_k, L.Nq = 256, 512, 1000, 3000, 700
+    acc = 4 * 1000 * 128 * 4
+    vec = (2 * 4 * 768 * 4 + 255) // 256 * 256
+    assert lib.fa_bwd_general_workspace_size(ctypes.byref(L)) == (acc + 255) // 256 * 256 + 2 * vec
+    assert lib.fa_bwd_general_workspace_size(None) == 0
+    assert lib.fa_bwd_workspace_size(4, 16, 4096, 128) == lib.fa_bwd_general_workspace_size(
+        ctypes.byref(_dense_layout(fa, 4, 16, 16, 4096, 4096, 128)))
+
+
 def test_workspace_sizes(lib):
     assert lib.fa_fwd_workspace_size(1, 1, 128, 64, 0) == 0
     assert lib.fa_fwd_workspace_size(1, 1, 128, 64, 1) == 3 * 128 * 64 * 2
