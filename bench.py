@@ -172,9 +172,26 @@ class ClockSampler:
 def oracle_sample(w, heads: int, seed_offset: int = 0, fwd_only: bool = False):
     """fwd (+ bwd) of `heads` whole heads of the workload with the fp64 oracle.
     Returns (seconds, algorithmic FLOPs of the sample, description)."""
-    from oracle import attention_bwd, attention_fwd, attention_fwd_decode
+    from oracle import attention_bwd, attention_bwd_varlen, attention_fwd, attention_fwd_decode, attention_fwd_varlen
     shape1 = (1, 1, w.N, w.d)
     t_total, flops = 0.0, 0.0
+    if w.varlen:   # one head of one sequence of the batch per sample, lengths taken in turn
+        lens = w.seq_lengths()
+        used = []
+        for i in range(heads):
+            n = lens[(i + seed_offset) % len(lens)]
+            used.append(n)
+            seed = w.seed + 7919 * (i + 1 + seed_offset)
+            f = {x: inputs.to_f64(inputs.make_tensor(seed, x, (n, 1, w.d)), "bf16") for x in ("q", "k", "v", "do")}
+            cu = np.array([0, n])
+            t0 = time.perf_counter()
+            attention_fwd_varlen(f["q"], f["k"], f["v"], cu, cu, w.scale, w.causal)
+            if not fwd_only:
+                attention_bwd_varlen(f["q"], f["k"], f["v"], f["do"], cu, cu, w.scale, w.causal)
+            t_total += time.perf_counter() - t0
+            flops += (1.0 if fwd_only else 3.5) * 4.0 * n * n * w.d / (2 if w.causal else 1)
+        return t_total, flops, (f"{'fwd' if fwd_only else 'fwd+bwd'} of {heads} head(s) of packed sequences "
+                                f"of lengths {used} (d={w.d}), numpy float64 oracle")
     if w.lq:       # decode: one query head's lq positions against its cache
         for i in range(heads):
             seed = w.seed + 7919 * (i + 1 + seed_offset)
@@ -245,6 +262,7 @@ def is_fwd_only(args, w) -> bool:
 def workload_config(w, step: str, note: str):
     c = {"workload": f"{w.name}: B={w.B} H={w.H}" + (f" H_kv={w.kv_heads}" if w.kv_heads != w.H else "")
                      + (f" Lq={w.lq}" if w.lq else "")
+                     + (f" packed, lengths N/8..N, total {sum(w.seq_lengths())}" if w.varlen else "")
                      + f" N={w.N} d={w.d} {'causal' if w.causal else 'non-causal'}"
                      + (f" K*{w.k_scale:g}" if w.k_scale != 1.0 else ""),
          "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "step": step, "l2": note}
@@ -362,6 +380,136 @@ def run_decode(args, w, fa, torch, dist, world, rank, local_rank, dev):
         dist.destroy_process_group()
 
 
+def run_varlen(args, w, fa, torch, dist, world, rank, local_rank, dev):
+    """Packed variable-length batch: fa_fwd_general + fa_bwd_general over B sequences of mixed lengths."""
+    lens = w.seq_lengths()
+    total, H, Hkv, d = sum(lens), w.H, w.kv_heads, w.d
+    seed = w.seed + 100003 * rank
+    shapes = {"q": (total, H, d), "k": (total, Hkv, d), "v": (total, Hkv, d), "do": (total, H, d)}
+    host = {n: inputs.make_tensor(seed, n, shp, w.k_scale if n == "k" else 1.0) for n, shp in shapes.items()}
+    pinned = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in host}
+    pinned["cu"] = torch.from_numpy(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)).pin_memory()
+    dv_ = {n: pinned[n].to(dev) for n in pinned}
+    o = torch.empty(shapes["q"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((H, total), dtype=torch.float32, device=dev)
+    dq = torch.empty(shapes["q"], dtype=torch.bfloat16, device=dev)
+    dk, dvv = (torch.empty(shapes["k"], dtype=torch.bfloat16, device=dev) for _ in range(2))
+    L = fa.layout_packed(dv_["q"], dv_["k"], dv_["v"], o, dv_["cu"], dv_["cu"], max(lens), max(lens),
+                         dv_["do"], dq, dk, dvv)
+    ws = torch.empty(fa.fa_bwd_general_workspace_size(L), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fa.fa_fwd_general(dv_["q"], dv_["k"], dv_["v"], o, lse, L, w.causal, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        fa.fa_bwd_general(dv_["q"], dv_["k"], dv_["v"], o, lse, dv_["do"], dq, dk, dvv, L, w.causal, ws,
+                          stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    in_bytes = sum(x.nbytes for x in host.values())
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_get_device_status() != fa.FA_OK:
+        raise SystemExit("device status reported an error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    if fa.fa_get_device_status() != fa.FA_OK:
+        raise SystemExit("device status reported an error in the timed region")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    fwd_all = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_all = [e[1].elapsed_time(e[2]) for e in evs]
+    fwd_flops = w.fwd_flops()
+    bwd_flops = 2.5 * fwd_flops
+    value = world * (fwd_flops + bwd_flops) * args.steps / (elapsed_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    kernels = {}
+    for name, flops, ts, note in (("fa_fwd_kernel", fwd_flops, fwd_all, "fa_fwd_general: one kernel"),
+                                  ("fa_bwd_kernel", bwd_flops, bwd_all,
+                                   "fa_bwd_general: prepare, main and finish kernels timed together")):
+        tf = flops / (statistics.mean(ts) * 1e-3) / 1e12
+        kernels[name] = {"ms": statistics.mean(ts), "median_ms": statistics.median(ts), "min_ms": min(ts),
+                         "tflops": tf, "frac_of_measured_burst": tf / burst, "frac_of_measured_sustained": tf / sustained,
+                         "note": note}
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    achieved = kernels[dom]["tflops"]
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                "frac": achieved / burst, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "frac_of_sustained": achieved / sustained,
+                "flops_per_launch": fwd_flops if dom == "fa_fwd_kernel" else bwd_flops,
+                "traffic": committed_traffic(dom, w.name)}
+    e2e = None
+    if not args.no_e2e:
+        outs = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dvv}
+        host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in outs.items()}
+
+        def e2e_step():
+            for n in pinned:
+                dv_[n].copy_(pinned[n], non_blocking=True)
+            step()
+            for n, t in outs.items():
+                host_out[n].copy_(t, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * (fwd_flops + bwd_flops) * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in pinned.values()),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs.values()),
+               "ms_per_step": e_ms / args.e2e_steps}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, f, desc = oracle_sample(w, args.cpu_heads)
+        cpu = {"value": f / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc + f"; {secs:.1f} s"}
+    cfg = workload_config(w, "fwd+bwd", f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB per step), no flush")
+    cfg["seq_lengths"] = lens
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "frac_of_measured_burst_peak": value / world / burst,
+        "fwd_tflops": kernels["fa_fwd_kernel"]["tflops"], "bwd_tflops": kernels["fa_bwd_kernel"]["tflops"],
+        "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     w = inputs.WORKLOADS[args.workload]
@@ -389,6 +537,9 @@ def main():
     fa.load_library()
     if w.lq:
         run_decode(args, w, fa, torch, dist, world, rank, local_rank, dev)
+        return
+    if w.varlen:
+        run_varlen(args, w, fa, torch, dist, world, rank, local_rank, dev)
         return
 
     fwd_only = is_fwd_only(args, w)

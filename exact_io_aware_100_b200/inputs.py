@@ -40,6 +40,7 @@ class Workload:
     backward: bool = False
     h_kv: int = 0       # key/value heads (0: as many as query heads)
     lq: int = 0         # decoding: this many query positions against N cached keys (0: N queries)
+    varlen: bool = False  # packed batch of B sequences of seq_lengths() rows (N the longest)
 
     @property
     def kv_heads(self) -> int:
@@ -49,7 +50,21 @@ class Workload:
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
+    def seq_lengths(self) -> list:
+        """Rows of each sequence: N for fixed-length workloads; for a packed batch,
+        seeded lengths uniform in [N / 8, N] (ragged, not tile multiples), the first
+        one N itself."""
+        if not self.varlen:
+            return [self.N] * self.B
+        rng = np.random.default_rng([int(self.seed), 7])
+        lens = rng.integers(self.N // 8, self.N + 1, size=self.B)
+        lens[0] = self.N
+        return [int(x) for x in lens]
+
     def fwd_flops(self) -> float:
+        if self.varlen:
+            f = sum(4.0 * self.H * n * n * self.d for n in self.seq_lengths())
+            return f / 2 if self.causal else f
         if self.lq:
             # query i of the last lq positions sees N - lq + i + 1 keys when causal, all N otherwise
             keys = (self.lq * (self.N - self.lq) + self.lq * (self.lq + 1) // 2) if self.causal else self.lq * self.N
@@ -69,6 +84,8 @@ WORKLOADS = {
     "prefill_gqa": Workload("prefill_gqa", 2, 32, 8192, 128, True, "bf16", 2.0, 1006, False, 8),
     # decoding one token per sequence against an 8192-key cache, 32 query heads over 8 key/value heads
     "decode": Workload("decode", 16, 32, 8192, 128, True, "bf16", 1.0, 1007, False, 8, 1),
+    # a packed batch of 16 sequences of mixed lengths (up to 8192), causal
+    "varlen": Workload("varlen", 16, 32, 8192, 128, True, "bf16", 1.0, 1008, varlen=True),
 }
 
 

@@ -47,3 +47,12 @@ def test_sample_rows():
     r = inputs.sample_rows(3, 65536, 256)
     assert r[0] == 0 and r[-1] == 65535 and len(r) <= 256 and len(set(r)) == len(r)
     assert (np.diff(r) > 0).all()
+
+
+def test_varlen_lengths_and_flops():
+    w = inputs.WORKLOADS["varlen"]
+    lens = w.seq_lengths()
+    assert len(lens) == w.B and lens[0] == w.N and all(w.N // 8 <= n <= w.N for n in lens)
+    assert lens == w.seq_lengths() and len(set(lens)) > w.B // 2
+    assert w.fwd_flops() == sum(4 * w.H * n * n * w.d for n in lens) / 2
+    assert inputs.WORKLOADS["prefill"].seq_lengths() == [8192, 8192]
