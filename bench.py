@@ -255,8 +255,9 @@ def run_reference(args, w):
 
 
 def is_fwd_only(args, w) -> bool:
-    """The backward covers bf16 inputs (d = 64 and 128); fp32-input and decode workloads time the forward."""
-    return args.fwd_only or w.dtype != "bf16" or bool(w.lq)
+    """The backward covers bf16 inputs at d = 64 and 128; fp32-input, head-dim-256 and decode workloads time
+    the forward."""
+    return args.fwd_only or w.dtype != "bf16" or bool(w.lq) or w.d == 256
 
 
 def workload_config(w, step: str, note: str):

@@ -11,6 +11,7 @@
 
 #include "bwd_kernel.cuh"
 #include "decode_kernel.cuh"
+#include "fwd256_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace fa {
@@ -27,6 +28,7 @@ struct DevState {
   uint32_t* status = nullptr;
   int sms = 0;
   bool fwd_attr[2][2] = {}, bwd_attr[2][2] = {};   // [d == 128][packed]: attributes set, registers checked
+  bool fwd256_attr[2] = {};                        // [packed]
   bool dec_attr = false;
 };
 DevState g_dev[kMaxDevices];
@@ -76,11 +78,12 @@ fa_status check_sizes(int B, int H, int N, int d, float scale) {
 }
 
 // 4-D bf16 tensor map over [batch][head][row][d] with element strides st:
-// box {64 columns, 128 rows, 1 head, 1 batch entry}, 128-byte swizzle (the
-// layout the UMMA descriptors in the kernels expect).  Extents of 1 get a
+// box {64 columns, box_rows rows, 1 head, 1 batch entry}, 128-byte swizzle
+// (the layout the UMMA descriptors in the kernels expect).  Extents of 1 get a
 // harmless dense stride (the copy never steps along them); an extent of 0
 // rows is mapped as 1 row that no copy reads.
-bool make_map4(CUtensorMap* m, const void* base, int d, int rows, int heads, int batches, const fa_strides& st) {
+bool make_map4(CUtensorMap* m, const void* base, int d, int rows, int heads, int batches, const fa_strides& st,
+               int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   if (rows < 1) rows = 1;
@@ -90,7 +93,7 @@ bool make_map4(CUtensorMap* m, const void* base, int d, int rows, int heads, int
   cuuint64_t strides[3] = {rows > 1 ? static_cast<cuuint64_t>(st.row) * 2 : dense,
                            heads > 1 ? static_cast<cuuint64_t>(st.head) * 2 : dense,
                            batches > 1 ? static_cast<cuuint64_t>(st.batch) * 2 : dense};
-  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -143,7 +146,7 @@ fa_status check_layout(const fa_layout& L, bool bwd) {
     if (reinterpret_cast<uintptr_t>(L.cu_seqlens_q) % 4 || reinterpret_cast<uintptr_t>(L.cu_seqlens_k) % 4)
       return FA_ERR_ALIGN;
   }
-  if (L.d != 64 && L.d != 128) return FA_ERR_UNSUPPORTED;
+  if (L.d != 64 && L.d != 128 && (bwd || L.d != 256)) return FA_ERR_UNSUPPORTED;   // d = 256: forward only
   // every row index the kernels form stays below 2^31
   const long long qr = static_cast<long long>(batches(L)) * L.H * (packed(L) ? L.total_q : L.Nq);
   const long long pr = static_cast<long long>(L.B) * L.H * ((static_cast<long long>(L.Nq) + 127) / 128 * 128);
@@ -262,13 +265,55 @@ fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, 
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Head dim 256 (forward, bf16): one 128-row query tile per CTA, 64-key blocks.
+template <bool PACKED>
+fa_status launch_fwd256_t(DevState* ds, const void* q, const void* k, const void* v, void* o, float* lse,
+                          const fa_layout& L, float scale, int causal, cudaStream_t stream) {
+  using C = Fwd256Cfg;
+  if (!ds->fwd256_attr[PACKED]) {
+    if (cudaFuncSetAttribute(fa_fwd256_kernel<PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    ds->fwd256_attr[PACKED] = true;
+  }
+  CUtensorMap tq, tk, tv;
+  const int bq = batches(L);
+  if (!make_map4(&tq, q, 256, q_rows(L), L.H, bq, L.q, 128) || !make_map4(&tk, k, 256, k_rows(L), L.H_kv, bq, L.k, 64) ||
+      !make_map4(&tv, v, 256, k_rows(L), L.H_kv, bq, L.v, 64))
+    return FA_ERR_CUDA;
+  FwdArgs a;
+  a.o = o;
+  a.lse = lse;
+  a.status = ds->status;
+  a.L = seq_layout(L);
+  a.so = kstrides(L.o);
+  a.group = L.H / L.H_kv;
+  a.n_qt = (L.Nq + 127) / 128;
+  a.num_tiles = L.B * L.H * a.n_qt;
+  a.causal = causal ? 1 : 0;
+  a.o_f32 = 0;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.wait_limit_ns = kWaitLimitNs;
+  const int grid = a.num_tiles < ds->sms ? a.num_tiles : ds->sms;
+  fa_fwd256_kernel<PACKED><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status launch_fwd256(DevState* ds, const void* q, const void* k, const void* v, void* o, float* lse,
+                        const fa_layout& L, float scale, int causal, cudaStream_t stream) {
+  if (L.Nq == 0 || (packed(L) && L.total_q == 0)) return FA_OK;   // no query row: nothing to write
+  if (static_cast<long long>(L.B) * L.H * ((L.Nq + 127) / 128) >= (1LL << 31)) return FA_ERR_INVALID;
+  return packed(L) ? launch_fwd256_t<true>(ds, q, k, v, o, lse, L, scale, causal, stream)
+                   : launch_fwd256_t<false>(ds, q, k, v, o, lse, L, scale, causal, stream);
+}
+
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv, int N,
                    int d, float scale, int causal, fa_dtype dtype, void* ws, size_t ws_bytes, cudaStream_t stream) {
   fa_status st = check_sizes(B, H, N, d, scale);
   if (st != FA_OK) return st;
   if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID;
   if (H_kv != H && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;   // grouped heads: bf16 inputs only
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && !(d == 256 && dtype == FA_BF16)) return FA_ERR_UNSUPPORTED;
   if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
   const size_t need = fa_fwd_workspace_size(B, H, N, d, dtype);
@@ -296,6 +341,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   }
   const int of32 = dtype == FA_F32 ? 1 : 0;
   const fa_layout L = dense_layout(B, H, H_kv, N, d);
+  if (d == 256) return launch_fwd256(ds, qq, kk, vv, o, lse, L, scale, causal, stream);
   return d == 64 ? launch_fwd<64>(ds, qq, kk, vv, o, lse, L, scale, causal, of32, stream)
                  : launch_fwd<128>(ds, qq, kk, vv, o, lse, L, scale, causal, of32, stream);
 }
@@ -310,6 +356,7 @@ fa_status fwd_general_impl(const void* q, const void* k, const void* v, void* o,
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
   DevState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
+  if (L.d == 256) return launch_fwd256(ds, q, k, v, o, lse, L, scale, causal, stream);
   return L.d == 64 ? launch_fwd<64>(ds, q, k, v, o, lse, L, scale, causal, 0, stream)
                    : launch_fwd<128>(ds, q, k, v, o, lse, L, scale, causal, 0, stream);
 }

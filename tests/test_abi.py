@@ -67,6 +67,8 @@ def test_argument_validation_without_device(lib):
     b = lib.fa_bwd
     args = [P16] * 9
     assert b(*args, 1, 1, 128, 96, 0.125, 1, P16, 1 << 30, None) == 2              # bwd d=96
+    assert b(*args, 1, 1, 128, 256, 0.125, 1, P16, 1 << 30, None) == 2             # bwd d=256 (forward only)
+    assert g(P16, P16, P16, P16, P16, 1, 1, 128, 256, 0.125, 0, 1, P16, 1 << 30, None) == 2   # fp32 at d=256
     assert b(*args, 1, 1, 128, 128, 0.125, 1, None, 0, None) == 4                  # no workspace
     need = lib.fa_bwd_workspace_size(1, 1, 128, 128)
     assert b(*args, 1, 1, 128, 128, 0.125, 1, 256, need - 1, None) == 4           # too small
