@@ -28,8 +28,10 @@
  *    anything is launched.  A kernel whose internal wait gives up (a bug, or a
  *    device that stopped making progress) sets a device status word that
  *    fa_get_device_status() reports; outputs are then undefined.
- *  - Supported: d in {64, 128} for the forward and the backward (d == 128 for
- *    fa_decode);
+ *  - Supported: d in {64, 128} for the forward and the backward; d == 256 for
+ *    the bf16 forward only (fa_fwd, fa_fwd_gqa, fa_fwd_general: one 128-row
+ *    query tile per CTA, after the nearauto.com FlashAttention-2 digest's
+ *    "head dimensions up to 256"); d == 128 for fa_decode;
  *    1 <= N <= 2^24; B*H*N*d < 2^31 elements per tensor.
  */
 #ifndef FA_H
@@ -178,7 +180,7 @@ typedef struct {
 } fa_layout;
 
 /*
- * Forward with a general layout.  q, o: [batch][H][row][d] bf16 with strides
+ * Forward with a general layout (d in {64, 128, 256}).  q, o: [batch][H][row][d] bf16 with strides
  * layout->q, layout->o; k, v: [batch][H_kv][row][d] bf16.  lse (float, dense):
  * [B, H, Nq] for fixed lengths, [H, total_q] for packed sequences.  Strides
  * of axes longer than 1 must be positive multiples of 8 elements (16 bytes)
@@ -193,7 +195,7 @@ fa_status fa_fwd_general(const void* q, const void* k, const void* v, void* o, f
                          const fa_layout* layout, float scale, int causal, fa_stream_t stream);
 
 /*
- * Backward with a general layout: the exact gradients of fa_fwd_general.
+ * Backward with a general layout (d in {64, 128}): the exact gradients of fa_fwd_general.
  * Inputs q, k, v, o, dout (strides layout->q, k, v, o, dout) and lse from the
  * forward (its layout); outputs dq, dk, dv (strides layout->dq, dk, dv),
  * written, not accumulated; dk and dv of a shared head sum over its set.
