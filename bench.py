@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_BYTES = 126 * 2**20
 EX2_PER_CLK_PER_SM = 16      # MUFU ex2 rate measured on this GPU by a probe (16 lanes / clock / SM)
 MUFU_SHARE_OF_EXP = 5 / 8    # both kernels evaluate three of every eight exp2 pairs by polynomial
-KERNEL_SOURCES = ["exact_io_aware_100_b200/csrc/ptx.cuh", "exact_io_aware_100_b200/csrc/fwd_kernel.cuh",
-                  "exact_io_aware_100_b200/csrc/bwd_kernel.cuh"]
+KERNEL_SOURCES = ["exact_io_aware_100_b200/csrc/ptx.cuh", "exact_io_aware_100_b200/csrc/layout.cuh",
+                  "exact_io_aware_100_b200/csrc/fwd_kernel.cuh", "exact_io_aware_100_b200/csrc/bwd_kernel.cuh"]
 
 
 def parse_args():
@@ -88,6 +88,27 @@ def committed_traffic(kernel: str, workload: str):
     if not e or e.get("csrc_sha256") != kernel_source_hash() or e.get("workload") != workload:
         return None
     return e.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------- ranks
+def rank_seed(w, rank: int) -> int:
+    """Each rank generates its own batch (weak scaling: disjoint data, no collective on the data path)."""
+    return w.seed + 100003 * rank
+
+
+def max_over_ranks(x: float, dist, world: int, device) -> float:
+    """The job's time is the slowest rank's (device-timed on each rank, then a MAX all-reduce)."""
+    if world <= 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank_step: float, world: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: the work of every rank over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (ms * 1e-3) / 1e12
 
 
 # --------------------------------------------------------------------- clocks
@@ -278,7 +299,7 @@ def workload_config(w, step: str, note: str):
 def run_decode(args, w, fa, torch, dist, world, rank, local_rank, dev):
     """Decode workloads: fa_decode (split partials + merge) over a cache larger than L2; HBM bound."""
     B, H, Hkv, Lq, N, d = w.B, w.H, w.kv_heads, w.lq, w.N, w.d
-    seed = w.seed + 100003 * rank
+    seed = rank_seed(w, rank)
     shapes = {"q": (B, H, Lq, d), "k": (B, Hkv, N, d), "v": (B, Hkv, N, d)}
     host = {n: inputs.make_tensor(seed, n, shp) for n, shp in shapes.items()}
     pinned = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in host}
@@ -321,12 +342,9 @@ def run_decode(args, w, fa, torch, dist, world, rank, local_rank, dev):
     elapsed_ms = sum(step_ms) if flush is not None else t0.elapsed_time(t1)
     if fa.fa_get_device_status() != fa.FA_OK:
         raise SystemExit("device status reported a timeout in the timed region")
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, world, dev)
     flops = w.fwd_flops()
-    value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = job_tflops(flops, world, args.steps, elapsed_ms)
     peaks, peak_src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     dec_ms = statistics.mean(step_ms)
@@ -354,8 +372,8 @@ def run_decode(args, w, fa, torch, dist, world, rank, local_rank, dev):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        e2e = {"value": world * flops * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(a.elapsed_time(b), dist, world, dev)
+        e2e = {"value": job_tflops(flops, world, args.e2e_steps, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": sum(x.nbytes for x in host.values()),
                "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4, "ms_per_step": e_ms / args.e2e_steps}
     cpu = None
@@ -385,7 +403,7 @@ def run_varlen(args, w, fa, torch, dist, world, rank, local_rank, dev):
     """Packed variable-length batch: fa_fwd_general + fa_bwd_general over B sequences of mixed lengths."""
     lens = w.seq_lengths()
     total, H, Hkv, d = sum(lens), w.H, w.kv_heads, w.d
-    seed = w.seed + 100003 * rank
+    seed = rank_seed(w, rank)
     shapes = {"q": (total, H, d), "k": (total, Hkv, d), "v": (total, Hkv, d), "do": (total, H, d)}
     host = {n: inputs.make_tensor(seed, n, shp, w.k_scale if n == "k" else 1.0) for n, shp in shapes.items()}
     pinned = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in host}
@@ -433,15 +451,12 @@ def run_varlen(args, w, fa, torch, dist, world, rank, local_rank, dev):
     elapsed_ms = t0.elapsed_time(t1)
     if fa.fa_get_device_status() != fa.FA_OK:
         raise SystemExit("device status reported an error in the timed region")
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, world, dev)
     fwd_all = [e[0].elapsed_time(e[1]) for e in evs]
     bwd_all = [e[1].elapsed_time(e[2]) for e in evs]
     fwd_flops = w.fwd_flops()
     bwd_flops = 2.5 * fwd_flops
-    value = world * (fwd_flops + bwd_flops) * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = job_tflops(fwd_flops + bwd_flops, world, args.steps, elapsed_ms)
     peaks, peak_src = load_peaks()
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -481,11 +496,8 @@ def run_varlen(args, w, fa, torch, dist, world, rank, local_rank, dev):
         b.record(stream)
         torch.cuda.synchronize()
         e_ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * (fwd_flops + bwd_flops) * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e_ms, dist, world, dev)
+        e2e = {"value": job_tflops(fwd_flops + bwd_flops, world, args.e2e_steps, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in pinned.values()),
                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs.values()),
                "ms_per_step": e_ms / args.e2e_steps}
@@ -546,7 +558,7 @@ def main():
     fwd_only = is_fwd_only(args, w)
     B, H, N, d = w.B, w.H, w.N, w.d
     shape = (B, H, N, d)
-    seed = w.seed + 100003 * rank          # each rank its own batch
+    seed = rank_seed(w, rank)          # each rank its own batch
     names = ("q", "k", "v") if fwd_only else ("q", "k", "v", "do")
     f32_in = w.dtype == "f32"               # fp32 inputs go through fa_fwd_ex (cast to bf16 on the GPU)
     gqa = w.kv_heads != w.H
@@ -642,15 +654,12 @@ def main():
     main_ms = None if fwd_only else statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     prep_ms = None if fwd_only else statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     fin_ms = None if fwd_only else statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, world, dev)
 
     fwd_flops = w.fwd_flops()
     bwd_flops = 2.5 * fwd_flops
     step_flops = fwd_flops + (0.0 if fwd_only else bwd_flops)
-    value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = job_tflops(step_flops, world, args.steps, elapsed_ms)
     peaks, peak_src = load_peaks()
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
 
@@ -715,11 +724,8 @@ def main():
         b.record(stream)
         torch.cuda.synchronize()
         e_ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * step_flops * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e_ms, dist, world, dev)
+        e2e = {"value": job_tflops(step_flops, world, args.e2e_steps, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.e2e_steps}
 
