@@ -40,7 +40,8 @@ L2_BYTES = 126 * 2**20
 EX2_PER_CLK_PER_SM = 16      # MUFU ex2 rate measured on this GPU by a probe (16 lanes / clock / SM)
 MUFU_SHARE_OF_EXP = 5 / 8    # both kernels evaluate three of every eight exp2 pairs by polynomial
 KERNEL_SOURCES = ["exact_io_aware_100_b200/csrc/ptx.cuh", "exact_io_aware_100_b200/csrc/layout.cuh",
-                  "exact_io_aware_100_b200/csrc/fwd_kernel.cuh", "exact_io_aware_100_b200/csrc/bwd_kernel.cuh"]
+                  "exact_io_aware_100_b200/csrc/fwd_kernel.cuh", "exact_io_aware_100_b200/csrc/bwd_kernel.cuh",
+                  "exact_io_aware_100_b200/csrc/fwd256_kernel.cuh", "exact_io_aware_100_b200/csrc/fa_api.cu"]
 
 
 def parse_args():
@@ -84,8 +85,8 @@ def committed_traffic(kernel: str, workload: str):
         return None
     with open(path) as f:
         d = json.load(f)
-    e = d.get("kernels", {}).get(kernel)
-    if not e or e.get("csrc_sha256") != kernel_source_hash() or e.get("workload") != workload:
+    e = d.get("kernels", {}).get(f"{kernel}@{workload}")
+    if not e or e.get("csrc_sha256") != kernel_source_hash():
         return None
     return e.get("dram_bytes_per_launch")
 

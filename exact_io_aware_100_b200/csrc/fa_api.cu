@@ -177,6 +177,18 @@ SeqLayout seq_layout(const fa_layout& L) {
 
 Strides kstrides(const fa_strides& st) { return Strides{st.batch, st.head, st.row}; }
 
+// Causal forward tile order: query heads taken in groups whose keys and values
+// (at most Nk rows each, bf16) fit in about 48 MB of L2 together, so the CTAs
+// working on a group's tiles share them there; whole key/value-head sets.
+int fwd_heads_per_group(const fa_layout& L) {
+  const double kv_bytes = 4.0 * (L.Nk > 0 ? L.Nk : 1) * L.d;   // K and V of one key/value head
+  long long kv_heads = static_cast<long long>(48.0 * (1 << 20) / kv_bytes);
+  if (kv_heads < 1) kv_heads = 1;
+  const long long hg = kv_heads * (L.H / L.H_kv);
+  const long long bh_all = static_cast<long long>(L.B) * L.H;
+  return static_cast<int>(hg < bh_all ? hg : bh_all);
+}
+
 // 3-D bf16 tensor map over [BH][N][d]: box {64 columns, box_rows rows, 1 head},
 // 128-byte swizzle (the layout the UMMA descriptors in the kernels expect).
 bool make_map(CUtensorMap* m, const void* base, int d, int N, int BH, int box_rows) {
@@ -256,6 +268,7 @@ fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, 
   a.group = L.H / L.H_kv;
   a.n_qt = (L.Nq + 255) / 256;
   a.num_tiles = L.B * L.H * a.n_qt;
+  a.heads_per_group = fwd_heads_per_group(L);
   a.causal = causal ? 1 : 0;
   a.o_f32 = o_f32;
   a.scale_log2 = scale * 1.4426950408889634f;
@@ -290,6 +303,7 @@ fa_status launch_fwd256_t(DevState* ds, const void* q, const void* k, const void
   a.group = L.H / L.H_kv;
   a.n_qt = (L.Nq + 127) / 128;
   a.num_tiles = L.B * L.H * a.n_qt;
+  a.heads_per_group = fwd_heads_per_group(L);
   a.causal = causal ? 1 : 0;
   a.o_f32 = 0;
   a.scale_log2 = scale * 1.4426950408889634f;

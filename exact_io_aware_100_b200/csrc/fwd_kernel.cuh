@@ -44,8 +44,9 @@ struct FwdArgs {
   SeqLayout L;
   Strides so;           // element strides of o
   int group;            // query heads per key/value head (1: multi-head; H: multi-query)
-  int n_qt;             // ceil(L.Nq / 256)
+  int n_qt;             // query tiles per sequence: ceil(L.Nq / tile rows)
   int num_tiles;        // B * H * n_qt
+  int heads_per_group;  // causal tile order: heads whose K / V fit in L2 together
   int causal;
   int o_f32;
   float scale_log2;     // scale * log2(e)
@@ -81,15 +82,20 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
 };
 
-// Work tile t -> (sequence b, query head h, tile qt of 256 query rows).  Query
+// Work tile t -> (sequence b, query head h, tile qt of query rows).  Query
 // head h reads key/value head h / group (sets of consecutive query heads share
 // one: grouped-query attention; group = 1 is multi-head).
 __device__ __forceinline__ void fwd_decode_tile(const FwdArgs& a, int t, int& b, int& h, int& qt) {
   const int bh_all = a.L.B * a.L.H;
   int bh;
-  if (a.causal) {            // longest work first
-    qt = a.n_qt - 1 - t / bh_all;
-    bh = t % bh_all;
+  if (a.causal) {            // heads in groups whose K / V fit in L2 together; longest work first in a group
+    const int per_group = a.heads_per_group * a.n_qt;
+    const int g = t / per_group;
+    const int r = t - g * per_group;
+    const int h0 = g * a.heads_per_group;
+    const int gh = min(a.heads_per_group, bh_all - h0);
+    qt = a.n_qt - 1 - r / gh;
+    bh = h0 + r % gh;
   } else {                   // neighbouring CTAs share a head's K / V in L2
     bh = t / a.n_qt;
     qt = t % a.n_qt;
