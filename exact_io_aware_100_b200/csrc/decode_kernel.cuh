@@ -20,11 +20,14 @@
 //    rows are the N_q queries of every query head of the key/value head's set
 //    (at most 16 rows).  64-key tiles of K and V stream through a two-stage
 //    TMA ring (128-byte swizzle, so per-lane shared reads are conflict free).
-//    Per tile, every warp works whatever the row count: scores with one thread
-//    per (key, group of rows), the online softmax with one warp per row, and
-//    P.V with each warp taking 8 of the 64 keys for all rows (four output
-//    columns per lane), keeping a partial O over its keys that the warps sum
-//    once at the end of the split.  Writes the split's normalised partial O
+//    Per tile, every warp works whatever the row count: scores with four
+//    adjacent lanes per key (a quarter of d each, all rows, packed fp32x2
+//    FMAs, summed by two shuffles; each K element is read from shared memory
+//    once), the online softmax with one warp per row, and P.V with each warp
+//    taking 8 of the 64 keys for all rows (four output columns per lane),
+//    keeping a partial O over its keys that the warps sum once at the end of
+//    the split.  Decoding is bound by HBM, so the kernel is built to spend as
+//    few issue slots per byte as it can.  Writes the split's normalised partial O
 //    (fp32) and its lse (-inf when no key is visible);
 //  * fa_decode_merge_kernel:  one warp per query row, merges the splits.
 #pragma once
@@ -57,8 +60,13 @@ struct DecCfg {
   static constexpr int THREADS = 256;
   static constexpr int KREG = KT * 128;          // one 64-column swizzle region of a 64-row tile
   static constexpr int TILE = 2 * KREG;          // a 64 x 128 bf16 tile (16 KB)
-  static constexpr int OFF_Q = 0;                // fp32 [R_MAX][D]; reused to sum the warps' partial O
-  static constexpr int OFF_ST = R_MAX * D * 4;   // two stages of K then V
+  // fp32 query rows, each d-quarter padded by 16 B so the four quarters a warp
+  // reads at once sit in different banks; reused as [R_MAX][D] to sum the
+  // warps' partial O at the end
+  static constexpr int Q_QUARTER = 36;           // floats per d-quarter (32 + 4 padding)
+  static constexpr int Q_ROW = 4 * Q_QUARTER;    // floats per query row
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_ST = R_MAX * Q_ROW * 4;   // two stages of K then V (1 KB aligned)
   static constexpr int STAGE = 2 * TILE;
   static constexpr int OFF_S = OFF_ST + 2 * STAGE;          // fp32 [R_MAX][KT]: scores, then P
   static constexpr int OFF_ROW = OFF_S + R_MAX * KT * 4;    // fp32 [R_MAX]: alpha of the tile, then l
@@ -116,7 +124,7 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       const int hq = bhq0 + r / a.Lq, i = r % a.Lq;
       x = __bfloat162float(a.q[(static_cast<size_t>(hq) * a.Lq + i) * D + c]);
     }
-    sq[idx] = x;
+    sq[r * C::Q_ROW + (c >> 5) * C::Q_QUARTER + (c & 31)] = x;
   }
   __syncthreads();
   const WaitCtl ctl{abort_flag, a.status, a.wait_limit_ns};
@@ -140,15 +148,15 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const float c2 = a.scale_log2;
   // causal limit of row r: key positions <= lim are visible
   auto lim_of = [&](int r) { return a.causal ? a.Nk - a.Lq + r % a.Lq : a.Nk - 1; };
-  // scores: thread = (key sk, rows sr0, sr0 + 4, sr0 + 8, sr0 + 12)
-  const int sk = tid & (C::KT - 1), sr0 = tid >> 6;
+  // scores: thread = (key sk, quarter dq of d), lanes 4 sk .. 4 sk + 3 of a warp hold one key
+  const int sk = tid >> 2, dq = tid & 3;
   // softmax: warp w owns rows w and w + 8 (running max m and sum l)
   const int ra = warp, rb = warp + 8;
   float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
   // P.V: warp w takes keys 8w .. 8w + 7 of every tile; lane owns columns 4 lane .. 4 lane + 3
-  float acc[RM][4];
+  float2 acc01[RM], acc23[RM];          // columns 4 lane, 4 lane + 1 and 4 lane + 2, 4 lane + 3
 #pragma unroll
-  for (int r = 0; r < RM; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+  for (int r = 0; r < RM; ++r) acc01[r] = acc23[r] = make_float2(0.f, 0.f);
   const int pj = lane >> 1, pregion = pj >> 3, pc = pj & 7;
   bool ok = true;
   int t_fail = n_tiles;
@@ -157,38 +165,37 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (!__syncthreads_and(ok)) { ok = false; t_fail = t; break; }   // every thread agrees before using the stage
     const uint8_t* st = smem + C::OFF_ST + (t & 1) * C::STAGE;
     const int kt0 = k_begin + t * C::KT;
-    // ---- scores S[r][sk] for this thread's rows (row groups beyond R do nothing)
-    if (sr0 < R) {
-      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+    // ---- scores S[r][sk]: this lane's quarter of d for every row, then the quarters summed
+    {
+      const uint8_t* krow = st + (dq >> 1) * C::KREG + sk * 128;
+      float2 kf[16];                       // d = 32 dq + 2 m, 32 dq + 2 m + 1
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {        // 16-byte chunks along d
-        const uint4 w = *reinterpret_cast<const uint4*>(st + (j >> 3) * C::KREG + sk * 128 + (((j & 7) ^ (sk & 7)) << 4));
-        float kf[8];
-        const uint32_t kw[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw[e]));
-          kf[2 * e] = f.x;
-          kf[2 * e + 1] = f.y;
-        }
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int r = sr0 + 4 * g;
-          if (r < R) {                        // uniform across the warp
-            const float4 q0 = *reinterpret_cast<const float4*>(sq + r * D + 8 * j);
-            const float4 q1 = *reinterpret_cast<const float4*>(sq + r * D + 8 * j + 4);
-            float x = sacc[g];
-            x = fmaf(q0.x, kf[0], x); x = fmaf(q0.y, kf[1], x); x = fmaf(q0.z, kf[2], x); x = fmaf(q0.w, kf[3], x);
-            x = fmaf(q1.x, kf[4], x); x = fmaf(q1.y, kf[5], x); x = fmaf(q1.z, kf[6], x); x = fmaf(q1.w, kf[7], x);
-            sacc[g] = x;
-          }
-        }
+      for (int i = 0; i < 4; ++i) {
+        const uint4 w = *reinterpret_cast<const uint4*>(krow + ((((dq & 1) * 4 + i) ^ (sk & 7)) << 4));
+        kf[4 * i + 0] = bf16x2_to_float2(w.x);
+        kf[4 * i + 1] = bf16x2_to_float2(w.y);
+        kf[4 * i + 2] = bf16x2_to_float2(w.z);
+        kf[4 * i + 3] = bf16x2_to_float2(w.w);
       }
       const int pos = kt0 + sk;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int r = sr0 + 4 * g;
-        if (r < R) ss[r * C::KT + sk] = (pos < k_end && pos <= lim_of(r)) ? sacc[g] : -INFINITY;
+      for (int r = 0; r < RM; ++r) {
+        if (r < R) {                       // uniform across the CTA
+          const float4* qp = reinterpret_cast<const float4*>(sq + r * C::Q_ROW + dq * C::Q_QUARTER);
+          float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 qa = qp[2 * i], qb = qp[2 * i + 1];
+            a0 = ffma2(make_float2(qa.x, qa.y), kf[4 * i + 0], a0);
+            a1 = ffma2(make_float2(qa.z, qa.w), kf[4 * i + 1], a1);
+            a0 = ffma2(make_float2(qb.x, qb.y), kf[4 * i + 2], a0);
+            a1 = ffma2(make_float2(qb.z, qb.w), kf[4 * i + 3], a1);
+          }
+          float x = (a0.x + a0.y) + (a1.x + a1.y);
+          x += __shfl_xor_sync(0xffffffffu, x, 1);
+          x += __shfl_xor_sync(0xffffffffu, x, 2);
+          if (dq == 0) ss[r * C::KT + sk] = (pos < k_end && pos <= lim_of(r)) ? x : -INFINITY;
+        }
       }
     }
     __syncthreads();
@@ -225,23 +232,32 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     for (int r = 0; r < RM; ++r) {
       if (r < R) {
         const float al = srow[r];
-        acc[r][0] *= al; acc[r][1] *= al; acc[r][2] *= al; acc[r][3] *= al;
+        acc01[r] = fmul2(acc01[r], make_float2(al, al));
+        acc23[r] = fmul2(acc23[r], make_float2(al, al));
       }
     }
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const int k = 8 * warp + kk;
-      const uint2 w = *reinterpret_cast<const uint2*>(vbase + k * 128 + ((pc ^ (k & 7)) << 4));
-      const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
-      const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+    for (int half = 0; half < 2; ++half) {   // keys 8 warp + 4 half .. + 3
+      float2 v01[4], v23[4];
+#pragma unroll
+      for (int kq = 0; kq < 4; ++kq) {
+        const int k = 8 * warp + 4 * half + kq;
+        const uint2 w = *reinterpret_cast<const uint2*>(vbase + k * 128 + ((pc ^ (k & 7)) << 4));
+        v01[kq] = bf16x2_to_float2(w.x);
+        v23[kq] = bf16x2_to_float2(w.y);
+      }
 #pragma unroll
       for (int r = 0; r < RM; ++r) {
         if (r < R) {
-          const float p = ss[r * C::KT + k];
-          acc[r][0] = fmaf(p, v01.x, acc[r][0]);
-          acc[r][1] = fmaf(p, v01.y, acc[r][1]);
-          acc[r][2] = fmaf(p, v23.x, acc[r][2]);
-          acc[r][3] = fmaf(p, v23.y, acc[r][3]);
+          const float4 p = *reinterpret_cast<const float4*>(ss + r * C::KT + 8 * warp + 4 * half);
+          acc01[r] = ffma2(make_float2(p.x, p.x), v01[0], acc01[r]);
+          acc23[r] = ffma2(make_float2(p.x, p.x), v23[0], acc23[r]);
+          acc01[r] = ffma2(make_float2(p.y, p.y), v01[1], acc01[r]);
+          acc23[r] = ffma2(make_float2(p.y, p.y), v23[1], acc23[r]);
+          acc01[r] = ffma2(make_float2(p.z, p.z), v01[2], acc01[r]);
+          acc23[r] = ffma2(make_float2(p.z, p.z), v23[2], acc23[r]);
+          acc01[r] = ffma2(make_float2(p.w, p.w), v01[3], acc01[r]);
+          acc23[r] = ffma2(make_float2(p.w, p.w), v23[3], acc23[r]);
         }
       }
     }
@@ -265,8 +281,10 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 #pragma unroll
   for (int r = 0; r < RM; ++r) {
     if (r < R) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) atomicAdd(sq + r * D + 4 * lane + e, acc[r][e]);
+      atomicAdd(sq + r * D + 4 * lane + 0, acc01[r].x);
+      atomicAdd(sq + r * D + 4 * lane + 1, acc01[r].y);
+      atomicAdd(sq + r * D + 4 * lane + 2, acc23[r].x);
+      atomicAdd(sq + r * D + 4 * lane + 3, acc23[r].y);
     }
   }
   __syncthreads();
