@@ -112,6 +112,60 @@ def job_tflops(flops_per_rank_step: float, world: int, steps: int, ms: float) ->
     return world * flops_per_rank_step * steps / (ms * 1e-3) / 1e12
 
 
+# --------------------------------------------------------------------- end to end
+def pipelined_e2e(torch, dev, pinned_in: dict, buf0: dict, out_names, run, steps: int):
+    """Device-timed milliseconds per step of the end-to-end loop a user would run:
+    every step copies its inputs from pinned host memory, runs the attention calls
+    and copies its outputs back to pinned host memory.  Two device buffer sets let
+    the host->device copy of step s+1, the compute of step s and the device->host
+    copy of step s-1 run at once on three streams (PCIe is full duplex and the
+    copy engines are not the SMs); events keep each buffer set's uses in order.
+    run(buffers, stream) enqueues one step's calls on `stream`."""
+    bufs = [buf0, {n: torch.empty_like(t) for n, t in buf0.items()}]
+    host_out = [{n: torch.empty(buf0[n].shape, dtype=buf0[n].dtype, pin_memory=True) for n in out_names}
+                for _ in range(2)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    cmp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+
+    def one(s):
+        b = s & 1
+        if s >= 2:
+            s_in.wait_event(cmp_done[b])           # step s-2's compute is done with these inputs
+        with torch.cuda.stream(s_in):
+            for n, t in pinned_in.items():
+                bufs[b][n].copy_(t, non_blocking=True)
+        in_ready[b].record(s_in)
+        s_cmp.wait_event(in_ready[b])
+        if s >= 2:
+            s_cmp.wait_event(out_done[b])          # step s-2's outputs have been copied out
+        run(bufs[b], s_cmp)
+        cmp_done[b].record(s_cmp)
+        s_out.wait_event(cmp_done[b])
+        with torch.cuda.stream(s_out):
+            for n in out_names:
+                host_out[b][n].copy_(bufs[b][n], non_blocking=True)
+        out_done[b].record(s_out)
+
+    for s in range(2):                             # untimed: first use of every buffer and stream
+        one(s)
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for s in range(2, 2 + steps):
+        one(s)
+    s_in.wait_event(out_done[0])
+    s_in.wait_event(out_done[1])
+    end.record(s_in)
+    torch.cuda.synchronize(dev)
+    return start.elapsed_time(end) / steps
+
+
+PIPELINE_NOTE = ("two device buffer sets; each step's host->device input copy, compute and device->host output "
+                 "copy on three streams, overlapping the neighbouring steps")
+
+
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML during the timed region."""
@@ -312,12 +366,14 @@ def run_decode(args, w, fa, torch, dist, world, rank, local_rank, dev):
     io_bytes = sum(x.nbytes for x in host.values()) + o.numel() * 2 + lse.numel() * 4
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if io_bytes < 2 * L2_BYTES else None
 
-    def step(ev=None):
+    buf0 = {"q": dv_["q"], "k": dv_["k"], "v": dv_["v"], "o": o, "lse": lse}
+
+    def step(ev=None, bf=buf0, st=stream):
         if ev is not None:
-            ev[0].record(stream)
-        fa.fa_decode(dv_["q"], dv_["k"], dv_["v"], o, lse, w.causal, ws, stream=stream)
+            ev[0].record(st)
+        fa.fa_decode(bf["q"], bf["k"], bf["v"], bf["o"], bf["lse"], w.causal, ws, stream=st)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(st)
 
     for _ in range(args.warmup):
         step()
@@ -355,28 +411,14 @@ def run_decode(args, w, fa, torch, dist, world, rank, local_rank, dev):
                 "bytes_per_launch": io_bytes, "traffic": None}
     e2e = None
     if not args.no_e2e:
-        host_out = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
-                    "lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)}
-
-        def e2e_step():
-            for n in host:
-                dv_[n].copy_(pinned[n], non_blocking=True)
-            step()
-            host_out["o"].copy_(o, non_blocking=True)
-            host_out["lse"].copy_(lse, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e_ms = max_over_ranks(a.elapsed_time(b), dist, world, dev)
-        e2e = {"value": job_tflops(flops, world, args.e2e_steps, e_ms), "unit": "TFLOP/s",
+        if world > 1:
+            dist.barrier()
+        e_ms = pipelined_e2e(torch, dev, pinned, buf0, ("o", "lse"), lambda bf, st: step(bf=bf, st=st),
+                             args.e2e_steps)
+        e_ms = max_over_ranks(e_ms, dist, world, dev)
+        e2e = {"value": job_tflops(flops, world, 1, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": sum(x.nbytes for x in host.values()),
-               "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4, "ms_per_step": e_ms / args.e2e_steps}
+               "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4, "ms_per_step": e_ms, "pipelined": PIPELINE_NOTE}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         secs, f, desc = oracle_sample(w, args.cpu_heads)
@@ -414,21 +456,24 @@ def run_varlen(args, w, fa, torch, dist, world, rank, local_rank, dev):
     lse = torch.empty((H, total), dtype=torch.float32, device=dev)
     dq = torch.empty(shapes["q"], dtype=torch.bfloat16, device=dev)
     dk, dvv = (torch.empty(shapes["k"], dtype=torch.bfloat16, device=dev) for _ in range(2))
-    L = fa.layout_packed(dv_["q"], dv_["k"], dv_["v"], o, dv_["cu"], dv_["cu"], max(lens), max(lens),
-                         dv_["do"], dq, dk, dvv)
-    ws = torch.empty(fa.fa_bwd_general_workspace_size(L), dtype=torch.uint8, device=dev)
+    L0 = fa.layout_packed(dv_["q"], dv_["k"], dv_["v"], o, dv_["cu"], dv_["cu"], max(lens), max(lens),
+                          dv_["do"], dq, dk, dvv)
+    ws = torch.empty(fa.fa_bwd_general_workspace_size(L0), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    buf0 = dict(dv_, o=o, lse=lse, dq=dq, dk=dk, dv=dvv)
 
-    def step(ev=None):
+    def step(ev=None, bf=buf0, st=stream):
+        L = L0 if bf is buf0 else fa.layout_packed(bf["q"], bf["k"], bf["v"], bf["o"], bf["cu"], bf["cu"], max(lens),
+                                                     max(lens), bf["do"], bf["dq"], bf["dk"], bf["dv"])
         if ev is not None:
-            ev[0].record(stream)
-        fa.fa_fwd_general(dv_["q"], dv_["k"], dv_["v"], o, lse, L, w.causal, stream=stream)
+            ev[0].record(st)
+        fa.fa_fwd_general(bf["q"], bf["k"], bf["v"], bf["o"], bf["lse"], L, w.causal, stream=st)
         if ev is not None:
-            ev[1].record(stream)
-        fa.fa_bwd_general(dv_["q"], dv_["k"], dv_["v"], o, lse, dv_["do"], dq, dk, dvv, L, w.causal, ws,
-                          stream=stream)
+            ev[1].record(st)
+        fa.fa_bwd_general(bf["q"], bf["k"], bf["v"], bf["o"], bf["lse"], bf["do"], bf["dq"], bf["dk"], bf["dv"], L,
+                          w.causal, ws, stream=st)
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record(st)
 
     in_bytes = sum(x.nbytes for x in host.values())
     for _ in range(args.warmup):
@@ -478,30 +523,15 @@ def run_varlen(args, w, fa, torch, dist, world, rank, local_rank, dev):
                 "traffic": committed_traffic(dom, w.name)}
     e2e = None
     if not args.no_e2e:
-        outs = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dvv}
-        host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in outs.items()}
-
-        def e2e_step():
-            for n in pinned:
-                dv_[n].copy_(pinned[n], non_blocking=True)
-            step()
-            for n, t in outs.items():
-                host_out[n].copy_(t, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
+        outs = ("o", "lse", "dq", "dk", "dv")
+        if world > 1:
+            dist.barrier()
+        e_ms = pipelined_e2e(torch, dev, pinned, buf0, outs, lambda bf, st: step(bf=bf, st=st), args.e2e_steps)
         e_ms = max_over_ranks(e_ms, dist, world, dev)
-        e2e = {"value": job_tflops(fwd_flops + bwd_flops, world, args.e2e_steps, e_ms), "unit": "TFLOP/s",
+        e2e = {"value": job_tflops(fwd_flops + bwd_flops, world, 1, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in pinned.values()),
-               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs.values()),
-               "ms_per_step": e_ms / args.e2e_steps}
+               "d2h_bytes_per_step": sum(buf0[n].numel() * buf0[n].element_size() for n in outs),
+               "ms_per_step": e_ms, "pipelined": PIPELINE_NOTE}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         secs, f, desc = oracle_sample(w, args.cpu_heads)
@@ -583,37 +613,41 @@ def main():
         ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     causal = w.causal
+    buf0 = dict(dv_, o=o, lse=lse)
+    if not fwd_only:
+        buf0.update(dq=dq, dk=dk, dv=dvv)
 
-    def step(ev=None):
+    def step(ev=None, bf=buf0, st=stream):
+        q_, k_, v_, o_, lse_ = bf["q"], bf["k"], bf["v"], bf["o"], bf["lse"]
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record(st)
         if f32_in:
-            fa.fa_fwd_ex(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, fa.FA_F32, fws, stream=stream)
+            fa.fa_fwd_ex(q_, k_, v_, o_, lse_, causal, fa.FA_F32, fws, stream=st)
         elif gqa:
-            fa.fa_fwd_gqa(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, stream=stream)
+            fa.fa_fwd_gqa(q_, k_, v_, o_, lse_, causal, stream=st)
         else:
-            fa.fa_fwd(dv_["q"], dv_["k"], dv_["v"], o, lse, causal, stream=stream)
+            fa.fa_fwd(q_, k_, v_, o_, lse_, causal, stream=st)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(st)
         if fwd_only:
             return
         if gqa:      # one call runs the three phases; its time is reported as the main kernel's
             if ev is not None:
-                ev[2].record(stream)
-            fa.fa_bwd_gqa(dv_["q"], dv_["k"], dv_["v"], o, lse, dv_["do"], dq, dk, dvv, causal, ws, stream=stream)
+                ev[2].record(st)
+            fa.fa_bwd_gqa(q_, k_, v_, o_, lse_, bf["do"], bf["dq"], bf["dk"], bf["dv"], causal, ws, stream=st)
             if ev is not None:
-                ev[3].record(stream)
-                ev[4].record(stream)
+                ev[3].record(st)
+                ev[4].record(st)
             return
-        fa.fa_bwd_prepare(o, lse, dv_["do"], ws, stream=stream)
+        fa.fa_bwd_prepare(o_, lse_, bf["do"], ws, stream=st)
         if ev is not None:
-            ev[2].record(stream)
-        fa.fa_bwd_main(dv_["q"], dv_["k"], dv_["v"], dv_["do"], dk, dvv, causal, ws, stream=stream)
+            ev[2].record(st)
+        fa.fa_bwd_main(q_, k_, v_, bf["do"], bf["dk"], bf["dv"], causal, ws, stream=st)
         if ev is not None:
-            ev[3].record(stream)
-        fa.fa_bwd_finish(dq, ws, stream=stream)
+            ev[3].record(st)
+        fa.fa_bwd_finish(bf["dq"], ws, stream=st)
         if ev is not None:
-            ev[4].record(stream)
+            ev[4].record(st)
 
     launches_per_step = (4 if f32_in else 1) if fwd_only else 4    # fp32: three cast kernels + the forward
     # Inputs and outputs smaller than twice L2 would stay cached between steps:
@@ -702,33 +736,16 @@ def main():
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
-        outs = {"o": o, "lse": lse} if fwd_only else {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dvv}
-        host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in outs.items()}
+        outs = ("o", "lse") if fwd_only else ("o", "lse", "dq", "dk", "dv")
         h2d = sum(pinned[n].numel() * pinned[n].element_size() for n in names)
-        d2h = sum(t.numel() * t.element_size() for t in outs.values())
-
-        def e2e_step():
-            for n in names:
-                dv_[n].copy_(pinned[n], non_blocking=True)
-            step()
-            for n, t in outs.items():
-                host_out[n].copy_(t, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d2h = sum(buf0[n].numel() * buf0[n].element_size() for n in outs)
         if world > 1:
             dist.barrier()
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
+        e_ms = pipelined_e2e(torch, dev, pinned, buf0, outs, lambda bf, st: step(bf=bf, st=st), args.e2e_steps)
         e_ms = max_over_ranks(e_ms, dist, world, dev)
-        e2e = {"value": job_tflops(step_flops, world, args.e2e_steps, e_ms), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e_ms / args.e2e_steps}
+        e2e = {"value": job_tflops(step_flops, world, 1, e_ms), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+               "pipelined": PIPELINE_NOTE}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
