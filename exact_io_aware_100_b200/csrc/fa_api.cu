@@ -674,8 +674,22 @@ fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float*
   if (Lq < 1 || Lq > Nk || H < 1 || H_kv > H || H % H_kv != 0 || 1LL * B * H * Lq * d >= (1LL << 31) ||
       B * H_kv > 65535)
     return FA_ERR_INVALID;
-  if (d != DecCfg::D || (H / H_kv) * Lq > DecCfg::R_MAX) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
+  if (d != DecCfg::D || (H / H_kv) * Lq > DecCfg::R_MAX) {
+    // outside the split-key decode kernel's shape (d = 128, at most 16 query rows per key/value
+    // head): the general forward computes the same result (N_q = Lq queries, bottom-right causal)
+    fa_layout L = {};
+    L.B = B;
+    L.H = H;
+    L.H_kv = H_kv;
+    L.d = d;
+    L.Nq = Lq;
+    L.Nk = Nk;
+    L.q = L.o = dense_strides(H, Lq, d);
+    L.k = L.v = dense_strides(H_kv, Nk, d);
+    return fwd_general_impl(q, k, v, o, lse, &L, scale, causal, static_cast<cudaStream_t>(stream));
+  }
   const size_t need = fa_decode_workspace_size(B, H, H_kv, Lq, Nk, d);
   if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return FA_ERR_WORKSPACE;

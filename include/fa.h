@@ -220,11 +220,13 @@ size_t fa_bwd_general_workspace_size(const fa_layout* layout);
  *  q, o: [B,H,Lq,d] bf16;  k, v: [B,H_kv,Nk,d] bf16 (H a multiple of H_kv, as
  *  in fa_fwd_gqa);  lse: [B,H,Lq] float (natural log).
  *  causal != 0: query i sees keys j <= Nk - Lq + i (bottom-right alignment).
- * Needs d == 128 and (H / H_kv) * Lq <= 16 (FA_ERR_UNSUPPORTED otherwise),
- * 1 <= Lq <= Nk and B * H_kv <= 65535 (FA_ERR_INVALID).  workspace: at least
+ * d in {64, 128, 256} (FA_ERR_UNSUPPORTED otherwise), 1 <= Lq <= Nk and
+ * B * H_kv <= 65535 (FA_ERR_INVALID).  workspace: at least
  * fa_decode_workspace_size(...) bytes, 256-byte aligned (the per-split partial
  * outputs); same layout, ownership, alignment, stream and error rules as
- * fa_fwd otherwise.  Two kernels: the split partials, then the merge.
+ * fa_fwd otherwise.  With d == 128 and (H / H_kv) * Lq <= 16 two kernels run:
+ * the split partials, then the merge; other shapes run the general forward
+ * (fa_fwd_general with N_q = Lq), which computes the same result.
  */
 fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                     int B, int H, int H_kv, int Lq, int Nk, int d, float scale, int causal,

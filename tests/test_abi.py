@@ -92,8 +92,7 @@ def test_decode_validation_without_device(lib):
     f = lib.fa_decode
     ok = (P16, P16, P16, P16, P16)
     assert f(*ok, 2, 8, 2, 1, 1000, 128, 0.088, 1, None, 0, None) == 4             # no workspace
-    assert f(*ok, 2, 8, 2, 1, 1000, 64, 0.125, 1, P16, 1 << 30, None) == 2        # d = 64
-    assert f(*ok, 2, 32, 1, 1, 1000, 128, 0.088, 1, P16, 1 << 30, None) == 2      # 32 rows in one set
+    assert f(*ok, 2, 8, 2, 1, 1000, 96, 0.125, 1, P16, 1 << 30, None) == 2        # d = 96
     assert f(*ok, 2, 8, 3, 1, 1000, 128, 0.088, 1, P16, 1 << 30, None) == 1       # uneven sets
     assert f(*ok, 2, 8, 2, 9, 8, 128, 0.088, 1, P16, 1 << 30, None) == 1          # more queries than keys
     assert f(*ok, 2, 8, 2, 0, 8, 128, 0.088, 1, P16, 1 << 30, None) == 1          # no query

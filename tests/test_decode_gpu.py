@@ -66,3 +66,27 @@ def test_decode_of_the_whole_sequence_matches_the_forward():
     torch.cuda.synchronize()
     assert_close("O", to_f64(o1), to_f64(o2))
     assert_lse(to_f64(l1), to_f64(l2).astype(np.float64))
+
+
+@pytest.mark.parametrize("B,H,H_kv,Lq,Nk,d,causal", [
+    (2, 32, 1, 1, 1000, 128, True),     # 32 query rows per key/value head: beyond the split-key kernel
+    (1, 8, 2, 4, 700, 64, True),        # head dim 64
+    (1, 4, 4, 3, 500, 256, False),      # head dim 256
+    (1, 4, 2, 9, 300, 256, True),
+])
+def test_decode_other_shapes_match_oracle(B, H, H_kv, Lq, Nk, d, causal):
+    """Shapes the split-key kernel does not take run the general forward; same result."""
+    import torch
+    import exact_io_aware_100_b200 as fa
+    seed = 3300 + Lq + d
+    host = {"q": inputs.make_tensor(seed, "q", (B, H, Lq, d)),
+            "k": inputs.make_tensor(seed, "k", (B, H_kv, Nk, d)),
+            "v": inputs.make_tensor(seed, "v", (B, H_kv, Nk, d))}
+    f64 = {n: inputs.to_f64(x, "bf16") for n, x in host.items()}
+    q, k, v = (to_device(host[n], "bf16") for n in ("q", "k", "v"))
+    o, lse = fa.decode(q, k, v, causal)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == fa.FA_OK
+    ro, rl = attention_fwd_decode(f64["q"], f64["k"], f64["v"], 1.0 / np.sqrt(d), causal)
+    assert_close("O", to_f64(o), ro)
+    assert_lse(to_f64(lse), rl)
