@@ -513,9 +513,12 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   a.bh_kv = L.B * L.H_kv;
   a.group = L.H / L.H_kv;
   a.n_kb = (L.Nk + 127) / 128;
-  // enough key/value heads per scheduling group to fill the GPU about twice over with key blocks
+  // Scheduling groups of key/value heads: enough query heads' key blocks to fill the GPU about
+  // twice over, counted in query heads, because a key/value head's items walk every query head of
+  // its set; the group's Q, dO and fp32 dQ accumulators (8 bytes per element at d = 128) then stay
+  // within L2 (e.g. 5 query heads of 8192 rows: 40 MB)
   const int nkb = a.n_kb < 1 ? 1 : a.n_kb;
-  const int want = (2 * ds->sms + nkb - 1) / nkb;
+  const int want = (2 * ds->sms + nkb - 1) / nkb / a.group;
   a.heads_per_group = want < 1 ? 1 : (want > a.bh_kv ? a.bh_kv : want);
   a.causal = causal ? 1 : 0;
   a.scale = scale;
