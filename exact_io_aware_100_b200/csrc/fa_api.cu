@@ -514,11 +514,12 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   a.group = L.H / L.H_kv;
   a.n_kb = (L.Nk + 127) / 128;
   // Scheduling groups of key/value heads: enough query heads' key blocks to fill the GPU about
-  // twice over, counted in query heads, because a key/value head's items walk every query head of
-  // its set; the group's Q, dO and fp32 dQ accumulators (8 bytes per element at d = 128) then stay
-  // within L2 (e.g. 5 query heads of 8192 rows: 40 MB)
+  // four times over, counted in query heads, because a key/value head's items walk every query
+  // head of its set; the group's Q, dO and fp32 dQ accumulators (8 bytes per element at d = 128)
+  // then stay within L2 (e.g. 9 query heads of 8192 rows: 75 MB).  Measured against one and two
+  // fills: equal for multi-head attention, 6.5% faster than two with grouped heads.
   const int nkb = a.n_kb < 1 ? 1 : a.n_kb;
-  const int want = (2 * ds->sms + nkb - 1) / nkb / a.group;
+  const int want = (4 * ds->sms + nkb - 1) / nkb / a.group;
   a.heads_per_group = want < 1 ? 1 : (want > a.bh_kv ? a.bh_kv : want);
   a.causal = causal ? 1 : 0;
   a.scale = scale;
