@@ -649,7 +649,7 @@ def main():
         if ev is not None:
             ev[4].record(st)
 
-    launches_per_step = (4 if f32_in else 1) if fwd_only else 4    # fp32: three cast kernels + the forward
+    launches_per_step = (2 if f32_in else 1) if fwd_only else 4    # fp32: one cast kernel (q, k, v) + the forward
     # Inputs and outputs smaller than twice L2 would stay cached between steps:
     # then every timed step is preceded by a write of a buffer larger than L2,
     # outside the kernels' events, and the step time is the sum of its events.
@@ -705,7 +705,7 @@ def main():
                                  "frac_of_measured_sustained": fwd_tf / sustained,
                                  "frac_of_datasheet": fwd_tf / DATASHEET_BF16_TFLOPS}}
     if f32_in:
-        kernels["fa_fwd_kernel"]["note"] = "fa_fwd_ex(FA_F32): three cast kernels + the forward"
+        kernels["fa_fwd_kernel"]["note"] = "fa_fwd_ex(FA_F32): one cast kernel (q, k, v) + the forward"
     if not fwd_only:
         main_tf = bwd_flops / (main_ms * 1e-3) / 1e12
         kernels["fa_bwd_kernel"] = {"ms": main_ms, "median_ms": statistics.median(main_all), "min_ms": min(main_all),

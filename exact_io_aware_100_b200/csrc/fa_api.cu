@@ -204,7 +204,14 @@ bool make_map(CUtensorMap* m, const void* base, int d, int N, int BH, int box_ro
   return r == CUDA_SUCCESS;
 }
 
-__global__ void cast_f32_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, size_t n4) {
+// q, k and v (blockIdx.y) rounded to bf16 in one launch: each is n4 float4 groups.
+struct CastArgs {
+  const float4* src[3];
+  uint2* dst[3];
+};
+__global__ void cast_f32_bf16_kernel(const CastArgs a, size_t n4) {
+  const float4* __restrict__ src = a.src[blockIdx.y];
+  uint2* __restrict__ dst = a.dst[blockIdx.y];
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const float4 v = src[i];
@@ -342,12 +349,14 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     const size_t part = round256(n * 2);
     uint8_t* w = static_cast<uint8_t*>(ws);
     const void* src[3] = {q, k, v};
+    CastArgs ca;
     for (int i = 0; i < 3; ++i) {
-      const size_t n4 = n / 4;
-      const int blocks = static_cast<int>((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
-      cast_f32_bf16_kernel<<<blocks, 256, 0, stream>>>(static_cast<const float4*>(src[i]),
-                                                        reinterpret_cast<uint2*>(w + i * part), n4);
+      ca.src[i] = static_cast<const float4*>(src[i]);
+      ca.dst[i] = reinterpret_cast<uint2*>(w + i * part);
     }
+    const size_t n4 = n / 4;
+    const unsigned blocks = static_cast<unsigned>((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096);
+    cast_f32_bf16_kernel<<<dim3(blocks, 3), 256, 0, stream>>>(ca, n4);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     qq = w;
     kk = w + part;
