@@ -247,7 +247,7 @@ static_assert(2 * BwdCfg<128>::REGS_PDS + BwdCfg<128>::REGS_DRAIN + BwdCfg<128>:
 // heads_per_group; inside a group the key blocks with the most query blocks
 // come first (causal), so the dQ accumulators being added to at any time are
 // those of a few heads and stay in L2.
-__device__ __forceinline__ void bwd_decode(const BwdArgs& a, int x, int& bh, int& kb) {   // bh: b * H_kv + h_kv
+__host__ __device__ __forceinline__ void bwd_decode(const BwdArgs& a, int x, int& bh, int& kb) {   // bh: b * H_kv + h_kv
   const int per_group = a.heads_per_group * a.n_kb;
   const int g = x / per_group;
   const int r = x - g * per_group;

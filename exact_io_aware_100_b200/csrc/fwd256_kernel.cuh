@@ -60,7 +60,7 @@ static_assert(Fwd256Cfg::SMEM_BYTES <= 232448, "shared memory plan");
 
 // Key blocks (64 keys) tile qt (128 rows) of sequence s reads; 0 when the tile
 // holds no query row or none of its rows sees a key.
-__device__ __forceinline__ int fwd256_num_kv(const FwdArgs& a, const SeqSpan& s, int qt) {
+__host__ __device__ __forceinline__ int fwd256_num_kv(const FwdArgs& a, const SeqSpan& s, int qt) {
   if (qt * 128 >= s.nq) return 0;
   const int n_all = (s.nk + 63) / 64;
   if (!a.causal) return n_all;

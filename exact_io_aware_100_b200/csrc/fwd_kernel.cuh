@@ -85,7 +85,7 @@ struct FwdCfg {
 // Work tile t -> (sequence b, query head h, tile qt of query rows).  Query
 // head h reads key/value head h / group (sets of consecutive query heads share
 // one: grouped-query attention; group = 1 is multi-head).
-__device__ __forceinline__ void fwd_decode_tile(const FwdArgs& a, int t, int& b, int& h, int& qt) {
+__host__ __device__ __forceinline__ void fwd_decode_tile(const FwdArgs& a, int t, int& b, int& h, int& qt) {
   const int bh_all = a.L.B * a.L.H;
   int bh;
   if (a.causal) {            // heads in groups whose K / V fit in L2 together; longest work first in a group
@@ -106,7 +106,7 @@ __device__ __forceinline__ void fwd_decode_tile(const FwdArgs& a, int t, int& b,
 
 // Key blocks (128 keys) tile qt of sequence s reads; 0 when the tile holds no
 // query row or none of its rows sees a key (then its rows are written as empty).
-__device__ __forceinline__ int fwd_num_kv(const FwdArgs& a, const SeqSpan& s, int qt) {
+__host__ __device__ __forceinline__ int fwd_num_kv(const FwdArgs& a, const SeqSpan& s, int qt) {
   if (qt * 256 >= s.nq) return 0;
   const int n_all = (s.nk + 127) / 128;
   if (!a.causal) return n_all;
