@@ -109,7 +109,13 @@ def _check(code: int, where: str) -> None:
 
 
 def _ptr(t) -> int | None:
-    return None if t is None else t.data_ptr()
+    """Device address of a CUDA tensor (None stays None).  Host tensors are refused here: the library
+    takes device pointers only and would otherwise launch kernels on host addresses."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor: the library reads and writes device memory only")
+    return t.data_ptr()
 
 
 def _stream(stream) -> int:
@@ -297,7 +303,7 @@ def layout_packed(q, k, v, o, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max
     if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
         raise ValueError("query and key offsets must both hold B + 1 entries")
     L = FaLayout(B=cu_seqlens_q.numel() - 1, H=H, H_kv=H_kv, d=d, Nq=int(max_seqlen_q), Nk=int(max_seqlen_k),
-                 cu_seqlens_q=cu_seqlens_q.data_ptr(), cu_seqlens_k=cu_seqlens_k.data_ptr(),
+                 cu_seqlens_q=_ptr(cu_seqlens_q), cu_seqlens_k=_ptr(cu_seqlens_k),
                  total_q=total_q, total_k=total_k)
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
         setattr(L, name, _strides_packed(t))

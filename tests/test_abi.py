@@ -190,3 +190,17 @@ def test_product_path_does_not_import_the_oracle():
     code = ("import sys, exact_io_aware_100_b200 as fa; fa.load_library(); "
             "assert not any(m == 'oracle' or m.startswith('oracle.') for m in sys.modules), 'oracle imported'")
     subprocess.run([sys.executable, "-c", code], check=True, cwd=ROOT)
+
+
+def test_binding_refuses_host_tensors(lib):
+    """Host (CPU) tensors never reach the library: it takes device pointers only."""
+    import torch
+    import exact_io_aware_100_b200 as fa
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward(q, q, q, True)
+    with pytest.raises(ValueError):
+        fa.forward(q.transpose(1, 2).contiguous().transpose(1, 2), q, q, True)
+    cu = torch.tensor([0, 128], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        fa.forward_varlen(q[0].transpose(0, 1), q[0].transpose(0, 1), q[0].transpose(0, 1), cu, cu, 128, 128, True)
