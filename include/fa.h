@@ -18,8 +18,11 @@
  * lengths; the general-layout calls below align it bottom-right).
  *
  * Conventions shared by every call:
- *  - Layout: q, k, v, o, dO, dq, dk, dv are dense row-major [B, H, N, d] with d
- *    innermost (element strides d, N*d, H*N*d).  lse is dense [B, H, N] float.
+ *  - Layout of the square calls (fa_fwd, fa_bwd, fa_fwd_ex, the phases,
+ *    fa_*_gqa, fa_bwd_noalloc): q, k, v, o, dO, dq, dk, dv are dense row-major
+ *    [B, H, N, d] with d innermost (element strides d, N*d, H*N*d); lse is
+ *    dense [B, H, N] float.  fa_fwd_general / fa_bwd_general take any lengths,
+ *    packed sequences and strides (fa_layout, below).
  *  - All pointers are DEVICE pointers owned by the caller; the library keeps
  *    no reference after the call returns and allocates nothing on these paths.
  *    Every pointer must be non-null and 16-byte aligned.
@@ -31,8 +34,9 @@
  *  - Supported: d in {64, 128} for the forward and the backward; d == 256 for
  *    the bf16 forward only (fa_fwd, fa_fwd_gqa, fa_fwd_general: one 128-row
  *    query tile per CTA, after the nearauto.com FlashAttention-2 digest's
- *    "head dimensions up to 256"); d == 128 for fa_decode;
- *    1 <= N <= 2^24; B*H*N*d < 2^31 elements per tensor.
+ *    "head dimensions up to 256"); fa_decode takes d in {64, 128, 256} (the
+ *    split-key kernel for d == 128); 1 <= N <= 2^24; B*H*N*d < 2^31
+ *    elements per tensor for the square calls.
  */
 #ifndef FA_H
 #define FA_H
@@ -46,7 +50,8 @@ extern "C" {
 
 typedef enum {
   FA_OK = 0,
-  FA_ERR_INVALID = 1,      /* bad sizes (B, H, N < 1, N too large, non-finite scale) */
+  FA_ERR_INVALID = 1,      /* bad sizes (B, H, N < 1, N too large, non-finite scale),
+                              or (device status) inconsistent packed sequence offsets */
   FA_ERR_UNSUPPORTED = 2,  /* d or dtype not supported by this call                 */
   FA_ERR_ALIGN = 3,        /* null or not 16-byte aligned pointer                     */
   FA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required              */
