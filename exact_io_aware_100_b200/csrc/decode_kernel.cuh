@@ -18,8 +18,11 @@
 //
 //  * fa_decode_kernel:  one CTA per (batch * key/value head, key split).  The
 //    rows are the N_q queries of every query head of the key/value head's set
-//    (at most 16 rows).  64-key tiles of K and V stream through a two-stage
-//    TMA ring (128-byte swizzle, so per-lane shared reads are conflict free).
+//    (at most 16 rows).  64-key tiles of K and V stream through a three-stage
+//    TMA ring (128-byte swizzle, so per-lane shared reads are conflict free);
+//    three block barriers per tile: the one that opens a tile also releases
+//    the previous tile's stage and score rows (its TMA reload is issued
+//    right after it).
 //    Per tile, every warp works whatever the row count: scores with four
 //    adjacent lanes per key (a quarter of d each, all rows, packed fp32x2
 //    FMAs, summed by two shuffles; each K element is read from shared memory
@@ -66,12 +69,13 @@ struct DecCfg {
   static constexpr int Q_QUARTER = 36;           // floats per d-quarter (32 + 4 padding)
   static constexpr int Q_ROW = 4 * Q_QUARTER;    // floats per query row
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_ST = R_MAX * Q_ROW * 4;   // two stages of K then V (1 KB aligned)
+  static constexpr int STAGES = 3;
+  static constexpr int OFF_ST = R_MAX * Q_ROW * 4;   // STAGES stages of K then V (1 KB aligned)
   static constexpr int STAGE = 2 * TILE;
-  static constexpr int OFF_S = OFF_ST + 2 * STAGE;          // fp32 [R_MAX][KT]: scores, then P
+  static constexpr int OFF_S = OFF_ST + STAGES * STAGE;     // fp32 [R_MAX][KT]: scores, then P
   static constexpr int OFF_ROW = OFF_S + R_MAX * KT * 4;    // fp32 [R_MAX]: alpha of the tile, then l
   static constexpr int OFF_BAR = OFF_ROW + R_MAX * 4;
-  static constexpr int OFF_MISC = OFF_BAR + 16;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * STAGES;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
 };
 
@@ -112,8 +116,7 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
   if (tid == 0) {
     *abort_flag = 0u;
-    mbar_init(b_full0, 1);
-    mbar_init(b_full0 + 8, 1);
+    for (int st = 0; st < C::STAGES; ++st) mbar_init(b_full0 + 8 * st, 1);
     fence_mbar_init();
   }
   // query rows (fp32), row r = (query head g of the set, position i); rows >= R are zero
@@ -128,9 +131,9 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   }
   __syncthreads();
   const WaitCtl ctl{abort_flag, a.status, a.wait_limit_ns};
-  auto issue = [&](int t) {         // tile t of this split into stage t % 2 (thread 0)
-    const uint32_t st = sbase + C::OFF_ST + (t & 1) * C::STAGE;
-    const uint32_t bar = b_full0 + 8 * (t & 1);
+  auto issue = [&](int t) {         // tile t of this split into stage t % STAGES (thread 0)
+    const uint32_t st = sbase + C::OFF_ST + (t % C::STAGES) * C::STAGE;
+    const uint32_t bar = b_full0 + 8 * (t % C::STAGES);
     mbar_expect_tx(bar, 2 * C::TILE);
     const int y = k_begin + t * C::KT;
     for (int r = 0; r < 2; ++r) {
@@ -139,8 +142,7 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     }
   };
   if (tid == 0) {
-    if (n_tiles > 0) issue(0);
-    if (n_tiles > 1) issue(1);
+    for (int t = 0; t < C::STAGES && t < n_tiles; ++t) issue(t);
   }
 
   float* ss = reinterpret_cast<float*>(smem + C::OFF_S);     // [R_MAX][KT]
@@ -161,9 +163,11 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   bool ok = true;
   int t_fail = n_tiles;
   for (int t = 0; t < n_tiles; ++t) {
-    ok = ok && mbar_wait(b_full0 + 8 * (t & 1), (t >> 1) & 1, ctl);
+    ok = ok && mbar_wait(b_full0 + 8 * (t % C::STAGES), (t / C::STAGES) & 1, ctl);
     if (!__syncthreads_and(ok)) { ok = false; t_fail = t; break; }   // every thread agrees before using the stage
-    const uint8_t* st = smem + C::OFF_ST + (t & 1) * C::STAGE;
+    // every thread is past tile t-1's P.V: its stage can be reloaded, its score rows rewritten
+    if (tid == 0 && t >= 1 && t - 1 + C::STAGES < n_tiles) issue(t - 1 + C::STAGES);
+    const uint8_t* st = smem + C::OFF_ST + (t % C::STAGES) * C::STAGE;
     const int kt0 = k_begin + t * C::KT;
     // ---- scores S[r][sk]: this lane's quarter of d for every row, then the quarters summed
     {
@@ -261,16 +265,16 @@ fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
       }
     }
-    __syncthreads();                       // stage t % 2 and the score rows are free again
-    if (tid == 0 && t + 2 < n_tiles) issue(t + 2);
   }
   if (!ok) {
-    // let the loads in flight (tiles t_fail and t_fail + 1) land before the CTA exits (bounded)
+    // let the loads in flight land before the CTA exits (bounded): tiles t_fail .. last issued
+    const int last_issued = C::STAGES - 1 + (t_fail > 1 ? t_fail - 1 : 0);
     if (tid == 0)
-      for (int t = t_fail; t < n_tiles && t < t_fail + 2; ++t)
-        mbar_wait_quiet(b_full0 + 8 * (t & 1), (t >> 1) & 1, 200000000ull);
+      for (int t = t_fail; t < n_tiles && t <= last_issued; ++t)
+        mbar_wait_quiet(b_full0 + 8 * (t % C::STAGES), (t / C::STAGES) & 1, 200000000ull);
     return;
   }
+  __syncthreads();                         // every warp is done with the last tile's P and alphas
   // ---- sum the warps' partial O (in the query buffer, which is no longer needed), then normalise
   for (int idx = tid; idx < C::R_MAX * D; idx += C::THREADS) sq[idx] = 0.f;
   if (lane == 0) {
