@@ -216,3 +216,15 @@ def test_varlen_rejects_bad_offsets():
     for cu_q, cu_k in (([0, 3, 5], [0, 4]), ([1, 5], [0, 4]), ([0, 6], [0, 4]), ([0, 4, 3, 5], [0, 1, 2, 4])):
         with pytest.raises(ValueError):
             attention_fwd_varlen(q, k, k, cu_q, cu_k, 1.0, False)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_head_dim_256_matches_torch_sdpa(causal):
+    """Head dimension 256 (the width the d = 256 kernel is checked at) against torch SDPA in float64."""
+    B, H, N, d = 1, 2, 40, 256
+    q, k, v = (_rand((B, H, N, d), 460 + i) for i in range(3))
+    o, lse = attention_fwd_general(q, k, v, d ** -0.5, causal)
+    to, tl, seen = _torch_ref(q, k, v, d ** -0.5, causal)
+    assert seen.all()
+    np.testing.assert_allclose(o, to, atol=1e-12)
+    np.testing.assert_allclose(lse, tl, atol=1e-12)
