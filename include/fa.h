@@ -242,7 +242,7 @@ size_t fa_decode_workspace_size(int B, int H, int H_kv, int Lq, int Nk, int d);
 
 /*
  * Backward without a caller-supplied workspace.  Same arguments, outputs and
- * numerics as fa_bwd, minus the workspace pair.  The paper has no counterpart
+ * numerics as fa_bwd, minus the workspace pair.  The pages have no counterpart
  * of this call; it exists for callers that cannot allocate device memory
  * themselves -- for example a plug-in whose host application owns every
  * device allocation through its own pool, or a serving path that must not

@@ -30,7 +30,7 @@ the softmax is two-pass (max, then exp / sum).  The only exception is
 ``attention_fwd_blockwise``, which deliberately takes the pages' tiled steps so
 that the merge identity can be pinned against the two-pass definition.
 
-Readings where the pages are silent or garbled (each is listed in the design doc):
+Readings where the pages are silent or garbled:
   * layout [B, H, N, d]: the pages' (batch, seq, d) with a head axis added;
   * lse is the natural log of sum_j exp(scale * q_i . k_j) over unmasked j;
   * causal masks j > i (top-left aligned, N_q == N_k);
