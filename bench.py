@@ -41,7 +41,8 @@ EX2_PER_CLK_PER_SM = 16      # MUFU ex2 rate measured on this GPU by a probe (16
 MUFU_SHARE_OF_EXP = 5 / 8    # both kernels evaluate three of every eight exp2 pairs by polynomial
 KERNEL_SOURCES = ["exact_io_aware_100_b200/csrc/ptx.cuh", "exact_io_aware_100_b200/csrc/layout.cuh",
                   "exact_io_aware_100_b200/csrc/fwd_kernel.cuh", "exact_io_aware_100_b200/csrc/bwd_kernel.cuh",
-                  "exact_io_aware_100_b200/csrc/fwd256_kernel.cuh", "exact_io_aware_100_b200/csrc/fa_api.cu"]
+                  "exact_io_aware_100_b200/csrc/fwd256_kernel.cuh", "exact_io_aware_100_b200/csrc/bwd256_kernel.cuh",
+                  "exact_io_aware_100_b200/csrc/fa_api.cu"]
 
 
 def parse_args():
@@ -56,6 +57,10 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-heads", type=int, default=6, help="heads in the CPU baseline sample")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the table of the other configurations (prefill workload only)")
+    p.add_argument("--sustained-s", type=float, default=3.0,
+                   help="seconds of back-to-back launches in the sustained leg (0 skips it)")
     p.add_argument("--shape", default=None,
                    help="B,H,N override of the workload's sizes (smaller cases for profiler captures)")
     return p.parse_args()
@@ -331,9 +336,8 @@ def run_reference(args, w):
 
 
 def is_fwd_only(args, w) -> bool:
-    """The backward covers bf16 inputs at d = 64 and 128; fp32-input, head-dim-256 and decode workloads time
-    the forward."""
-    return args.fwd_only or w.dtype != "bf16" or bool(w.lq) or w.d == 256
+    """The backward covers bf16 inputs (d = 64, 128, 256); fp32-input and decode workloads time the forward."""
+    return args.fwd_only or w.dtype != "bf16" or bool(w.lq)
 
 
 def workload_config(w, step: str, note: str):
@@ -552,6 +556,159 @@ def run_varlen(args, w, fa, torch, dist, world, rank, local_rank, dev):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------- the other configurations
+# The metric covers forward and backward, causal and non-causal, at every configuration the
+# workload list names.  The headline line measures the prefill configuration; this table adds the
+# others, measured the same way (CUDA events on the launching stream around each call, an L2 flush
+# before every step whose inputs and outputs fit in twice the L2), one after the other in the same
+# process.
+CONFIG_TABLE = (("1", "single_head", 20), ("2", "multi_head", 20), ("2c", "multi_head_causal", 20),
+                ("4", "long_context", 3), ("5", "backward", 10))
+
+
+def _device_inputs(torch, dev, w, names, seed):
+    shape = (w.B, w.H, w.N, w.d)
+    out = {}
+    for n in names:
+        x = inputs.make_tensor(seed, n, shape, w.k_scale if n == "k" else 1.0, "f32" if w.dtype == "f32" else "bf16")
+        t = torch.from_numpy(x) if w.dtype == "f32" else torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)
+        out[n] = t.to(dev)
+    return out
+
+
+def measure_config(fa, torch, dev, local_rank, w, steps: int, warmup: int, burst: float, sustained: float):
+    """Forward (and, for bf16 inputs, backward) of one configuration: TFLOP/s from the mean of the
+    per-call CUDA events, fractions of the measured and datasheet peaks, the NVML clock median."""
+    fwd_only = w.dtype != "bf16"
+    names = ("q", "k", "v") if fwd_only else ("q", "k", "v", "do")
+    t = _device_inputs(torch, dev, w, names, w.seed)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    o = torch.empty((B, H, N, d), dtype=torch.float32 if w.dtype == "f32" else torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    fws = None
+    if w.dtype == "f32":
+        fws = torch.empty(fa.fa_fwd_workspace_size(B, H, N, d, fa.FA_F32), dtype=torch.uint8, device=dev)
+    if not fwd_only:
+        dq, dk, dv = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+        ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        if w.dtype == "f32":
+            fa.fa_fwd_ex(t["q"], t["k"], t["v"], o, lse, w.causal, fa.FA_F32, fws, stream=stream)
+        else:
+            fa.fa_fwd(t["q"], t["k"], t["v"], o, lse, w.causal, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if fwd_only:
+            return
+        fa.fa_bwd_prepare(o, lse, t["do"], ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        fa.fa_bwd_main(t["q"], t["k"], t["v"], t["do"], dk, dv, w.causal, ws, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        fa.fa_bwd_finish(dq, ws, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    io_bytes = sum(x.numel() * x.element_size() for x in t.values()) * (1 if fwd_only else 2) + \
+        o.numel() * o.element_size()
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if io_bytes < 2 * L2_BYTES else None
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    with ClockSampler(local_rank, period_s=0.005) as clk:
+        for s in range(steps):
+            if flush is not None:
+                flush.fill_(s & 0xff)
+            step(evs[s])
+        torch.cuda.synchronize(dev)
+    if fa.fa_get_device_status() != fa.FA_OK:
+        raise SystemExit(f"device status reported an error in configuration {w.name}")
+    fwd_flops = w.fwd_flops()
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    fwd_tf = fwd_flops / (fwd_ms * 1e-3) / 1e12
+    r = {"workload": workload_config(w, "fwd" if fwd_only else "fwd+bwd", "")["workload"],
+         "steps": steps, "warmup": warmup,
+         "l2": "flushed before every step" if flush is not None else "inputs larger than L2, no flush",
+         "fwd_ms": fwd_ms, "fwd_tflops": fwd_tf, "fwd_frac_of_measured_burst": fwd_tf / burst,
+         "fwd_frac_of_measured_sustained": fwd_tf / sustained, "fwd_frac_of_datasheet": fwd_tf / DATASHEET_BF16_TFLOPS}
+    if w.dtype == "f32":
+        r["fwd_note"] = "fa_fwd_ex(FA_F32): one cast kernel (q, k, v) and the forward"
+        alg = 3 * B * H * N * d * 4 + B * H * N * d * 4 + 4 * B * H * N
+        r["fwd_us"] = fwd_ms * 1e3
+        r["fwd_algorithmic_gbs"] = alg / (fwd_ms * 1e-3) / 1e9
+    if not fwd_only:
+        bwd_flops = 2.5 * fwd_flops
+        bwd_ms = statistics.mean(e[1].elapsed_time(e[4]) for e in evs)
+        main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+        bwd_tf, main_tf = bwd_flops / (bwd_ms * 1e-3) / 1e12, bwd_flops / (main_ms * 1e-3) / 1e12
+        r.update({"bwd_ms": bwd_ms, "bwd_tflops": bwd_tf, "bwd_frac_of_measured_burst": bwd_tf / burst,
+                  "bwd_frac_of_datasheet": bwd_tf / DATASHEET_BF16_TFLOPS,
+                  "bwd_main_kernel_ms": main_ms, "bwd_main_kernel_tflops": main_tf,
+                  "bwd_main_kernel_frac_of_measured_burst": main_tf / burst})
+        step_tf = (fwd_flops + bwd_flops) / ((fwd_ms + bwd_ms) * 1e-3) / 1e12
+        r.update({"step_tflops": step_tf, "step_frac_of_measured_burst": step_tf / burst})
+    r["clocks"] = clk.summary()
+    return r
+
+
+def sustained_leg(fa, torch, dev, local_rank, w, seconds: float, sustained: float):
+    """The configuration's forward, then its whole step (forward + the three backward phases),
+    launched back to back on one stream for at least `seconds` each: device time from CUDA events
+    around the loop, the NVML median SM clock during it, and the fraction of the measured sustained
+    bf16 peak (the one a kernel meets inside a seconds-long run)."""
+    t = _device_inputs(torch, dev, w, ("q", "k", "v", "do"), w.seed)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        fa.fa_fwd(t["q"], t["k"], t["v"], o, lse, w.causal, stream=stream)
+
+    def full():
+        fwd()
+        fa.fa_bwd(t["q"], t["k"], t["v"], o, lse, t["do"], dq, dk, dv, w.causal, ws, stream=stream)
+
+    out = {}
+    fwd_flops = w.fwd_flops()
+    for name, fn, flops in (("fwd", fwd, fwd_flops), ("step", full, 3.5 * fwd_flops)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        iters = max(10, int(math.ceil(seconds * 1e3 / max(a.elapsed_time(b), 1e-3))))
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank, period_s=0.05) as clk:
+            t0.record(stream)
+            for _ in range(iters):
+                fn()
+            t1.record(stream)
+            torch.cuda.synchronize(dev)
+        ms = t0.elapsed_time(t1)
+        tf = flops * iters / (ms * 1e-3) / 1e12
+        out[name] = {"iterations": iters, "seconds": ms * 1e-3, "tflops": tf,
+                     "frac_of_measured_sustained": tf / sustained, "frac_of_datasheet": tf / DATASHEET_BF16_TFLOPS,
+                     "clocks": clk.summary()}
+    if fa.fa_get_device_status() != fa.FA_OK:
+        raise SystemExit("device status reported an error in the sustained leg")
+    out["workload"] = workload_config(w, "fwd+bwd", "")["workload"]
+    out["note"] = ("back-to-back launches on one stream for at least %.0f s each; tflops from CUDA events around "
+                   "the loop; clocks sampled by NVML during it" % seconds)
+    return out
 
 
 def main():
@@ -776,6 +933,21 @@ def main():
     line["exp"] = {"count_fwd": n_exp, "count_bwd": 0 if fwd_only else n_exp, "on_mufu": MUFU_SHARE_OF_EXP,
                    "mufu_time_share_fwd": mufu_s / (fwd_ms * 1e-3),
                    "mufu_time_share_bwd": None if fwd_only else mufu_s / (main_ms * 1e-3)}
+    if w.name == "prefill" and world == 1:
+        if not args.no_configs:    # the other configurations of the metric, same process, after the headline
+            table = {"3": {"workload": line["config"]["workload"], "fwd_tflops": fwd_tf,
+                           "fwd_frac_of_measured_burst": fwd_tf / burst,
+                           "bwd_tflops": line["bwd_tflops"], "bwd_main_kernel_tflops": kernels["fa_bwd_kernel"]["tflops"],
+                           "bwd_main_kernel_frac_of_measured_burst": kernels["fa_bwd_kernel"]["frac_of_measured_burst"],
+                           "note": "the headline measurement of this line", "clocks": line["clocks"]}}
+            del buf0, dv_
+            for key, name, n_steps in CONFIG_TABLE:
+                table[key] = measure_config(fa, torch, dev, local_rank, inputs.WORKLOADS[name], n_steps, 3, burst,
+                                            sustained)
+                torch.cuda.empty_cache()
+            line["configs"] = table
+        if args.sustained_s > 0:
+            line["sustained"] = sustained_leg(fa, torch, dev, local_rank, w, args.sustained_s, sustained)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

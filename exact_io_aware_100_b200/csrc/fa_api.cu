@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "bwd256_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "fwd256_kernel.cuh"
@@ -25,9 +26,11 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per bounded 
 
 struct DevState {
   bool ready = false;
+  unsigned long long ctx_id = 0;                   // context the state below was set up in
   uint32_t* status = nullptr;
   int sms = 0;
   bool fwd_attr[2][2] = {}, bwd_attr[2][2] = {};   // [d == 128][packed]: attributes set, registers checked
+  bool bwd256_attr[2] = {};                        // [packed]
   bool fwd256_attr[2] = {};                        // [packed]
   bool dec_attr = false;
 };
@@ -47,19 +50,52 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+}  // namespace
+
+// Unique id of the CUDA context current on this thread, 0 if there is none yet.
+// Device addresses of the library's __device__ arrays and the kernel attributes
+// belong to a context: after a device reset (a new primary context) they are
+// looked up and set again.
+unsigned long long current_ctx_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+namespace {
+
 fa_status device_state(DevState** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
   DevState& s = g_dev[dev];
-  if (!s.ready) {
+  if (!s.ready || s.ctx_id != current_ctx_id()) {
+    s = DevState();
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return FA_ERR_CUDA;   // makes the context current
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
       return FA_ERR_CUDA;
     s.status = static_cast<uint32_t*>(p);
     s.sms = sms;
+    s.ctx_id = current_ctx_id();
     s.ready = true;
   }
   *out = &s;
@@ -70,8 +106,12 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The score scale must be finite and positive: the kernels take the row
+// maximum of the unscaled scores as the softmax reference.
+bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.0f; }
+
 fa_status check_sizes(int B, int H, int N, int d, float scale) {
-  if (B < 1 || H < 1 || N < 1 || N > (1 << 24) || !std::isfinite(scale)) return FA_ERR_INVALID;
+  if (B < 1 || H < 1 || N < 1 || N > (1 << 24) || !scale_ok(scale)) return FA_ERR_INVALID;
   const long long numel = 1LL * B * H * N * d;
   if (numel >= (1LL << 31)) return FA_ERR_INVALID;
   return FA_OK;
@@ -146,7 +186,7 @@ fa_status check_layout(const fa_layout& L, bool bwd) {
     if (reinterpret_cast<uintptr_t>(L.cu_seqlens_q) % 4 || reinterpret_cast<uintptr_t>(L.cu_seqlens_k) % 4)
       return FA_ERR_ALIGN;
   }
-  if (L.d != 64 && L.d != 128 && (bwd || L.d != 256)) return FA_ERR_UNSUPPORTED;   // d = 256: forward only
+  if (L.d != 64 && L.d != 128 && L.d != 256) return FA_ERR_UNSUPPORTED;
   // every row index the kernels form stays below 2^31
   const long long qr = static_cast<long long>(batches(L)) * L.H * (packed(L) ? L.total_q : L.Nq);
   const long long pr = static_cast<long long>(L.B) * L.H * ((static_cast<long long>(L.Nq) + 127) / 128 * 128);
@@ -375,7 +415,7 @@ fa_status fwd_general_impl(const void* q, const void* k, const void* v, void* o,
   const fa_layout& L = *Lp;
   fa_status st = check_layout(L, false);
   if (st != FA_OK) return st;
-  if (!std::isfinite(scale)) return FA_ERR_INVALID;
+  if (!scale_ok(scale)) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
   DevState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
@@ -459,6 +499,16 @@ fa_status prepare_bwd_kernel() {
   return FA_OK;
 }
 
+template <bool PACKED>
+fa_status prepare_bwd256_kernel() {
+  if (!launch_regs_are(reinterpret_cast<const void*>(fa_bwd256_kernel<PACKED>), Bwd256Cfg::LAUNCH_REGS))
+    return FA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(fa_bwd256_kernel<PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Bwd256Cfg::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
 template <int D>
 void launch_bwd_main(bool pk, unsigned grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
@@ -475,7 +525,7 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
                    void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   fa_status st = check_layout(L, true);
   if (st != FA_OK) return st;
-  if (!std::isfinite(scale)) return FA_ERR_INVALID;
+  if (!scale_ok(scale)) return FA_ERR_INVALID;
   const int d = L.d;
   if ((phases & PH_PREPARE) && (!aligned16(o) || !aligned16(lse) || !aligned16(dout))) return FA_ERR_ALIGN;
   if ((phases & PH_MAIN) && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
@@ -488,7 +538,11 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   DevState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
   const bool pk = packed(L);
-  if ((phases & PH_MAIN) && !ds->bwd_attr[d == 128][pk]) {
+  if ((phases & PH_MAIN) && d == 256 && !ds->bwd256_attr[pk]) {
+    st = pk ? prepare_bwd256_kernel<true>() : prepare_bwd256_kernel<false>();
+    if (st != FA_OK) return st;
+    ds->bwd256_attr[pk] = true;
+  } else if ((phases & PH_MAIN) && d != 256 && !ds->bwd_attr[d == 128][pk]) {
     st = d == 64 ? (pk ? prepare_bwd_kernel<64, true>() : prepare_bwd_kernel<64, false>())
                  : (pk ? prepare_bwd_kernel<128, true>() : prepare_bwd_kernel<128, false>());
     if (st != FA_OK) return st;
@@ -527,8 +581,10 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   // head of its set; the group's Q, dO and fp32 dQ accumulators (8 bytes per element at d = 128)
   // then stay within L2 (e.g. 9 query heads of 8192 rows: 75 MB).  Measured against one and two
   // fills: equal for multi-head attention, 6.5% faster than two with grouped heads.
+  // (at d = 256 two CTAs share each key block, so a fill holds half as many blocks)
   const int nkb = a.n_kb < 1 ? 1 : a.n_kb;
-  const int want = (4 * ds->sms + nkb - 1) / nkb / a.group;
+  const int fills = d == 256 ? 2 * ds->sms : 4 * ds->sms;
+  const int want = (fills + nkb - 1) / nkb / a.group;
   a.heads_per_group = want < 1 ? 1 : (want > a.bh_kv ? a.bh_kv : want);
   a.causal = causal ? 1 : 0;
   a.scale = scale;
@@ -537,18 +593,29 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   if (phases & PH_PREPARE) {
     if (d == 64)
       fa_bwd_pre_kernel<64><<<ds->sms * 8, 256, 0, stream>>>(a);
-    else
+    else if (d == 128)
       fa_bwd_pre_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
+    else
+      fa_bwd_pre_kernel<256><<<ds->sms * 8, 256, 0, stream>>>(a);
   }
   if ((phases & PH_MAIN) && a.n_kb > 0 && !(packed(L) && L.total_k == 0)) {
     CUtensorMap tq, tk, tv, tdo;
     const int bq = batches(L);
-    if (!make_map4(&tq, q, d, q_rows(L), L.H, bq, L.q) || !make_map4(&tk, k, d, k_rows(L), L.H_kv, bq, L.k) ||
-        !make_map4(&tv, v, d, k_rows(L), L.H_kv, bq, L.v) || !make_map4(&tdo, dout, d, q_rows(L), L.H, bq, L.dout))
+    const int qbox = d == 256 ? Bwd256Cfg::BM : 128;   // rows of a query block
+    if (!make_map4(&tq, q, d, q_rows(L), L.H, bq, L.q, qbox) || !make_map4(&tk, k, d, k_rows(L), L.H_kv, bq, L.k) ||
+        !make_map4(&tv, v, d, k_rows(L), L.H_kv, bq, L.v) ||
+        !make_map4(&tdo, dout, d, q_rows(L), L.H, bq, L.dout, qbox))
       return FA_ERR_CUDA;
-    const long long grid = static_cast<long long>(a.n_kb) * a.bh_kv;
+    const long long grid = static_cast<long long>(a.n_kb) * a.bh_kv * (d == 256 ? 2 : 1);
     if (grid >= (1LL << 31)) return FA_ERR_INVALID;
-    if (d == 64)
+    if (d == 256) {
+      if (pk)
+        fa_bwd256_kernel<true><<<static_cast<unsigned>(grid), Bwd256Cfg::THREADS, Bwd256Cfg::SMEM_BYTES, stream>>>(
+            tq, tk, tv, tdo, a);
+      else
+        fa_bwd256_kernel<false><<<static_cast<unsigned>(grid), Bwd256Cfg::THREADS, Bwd256Cfg::SMEM_BYTES, stream>>>(
+            tq, tk, tv, tdo, a);
+    } else if (d == 64)
       launch_bwd_main<64>(pk, static_cast<unsigned>(grid), tq, tk, tv, tdo, a, stream);
     else
       launch_bwd_main<128>(pk, static_cast<unsigned>(grid), tq, tk, tv, tdo, a, stream);
@@ -556,8 +623,10 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
   if ((phases & PH_FINISH) && a.acc_rows > 0) {
     if (d == 64)
       fa_bwd_dq_kernel<64><<<ds->sms * 8, 256, 0, stream>>>(a);
-    else
+    else if (d == 128)
       fa_bwd_dq_kernel<128><<<ds->sms * 8, 256, 0, stream>>>(a);
+    else
+      fa_bwd_dq_kernel<256><<<ds->sms * 8, 256, 0, stream>>>(a);
   }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -620,18 +689,21 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[FA_NOALLOC_SCRATCH_BY
 
 namespace {
 void* g_noalloc_ptr[fa::kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[fa::kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-// Device address of g_noalloc_scratch on the current device (looked up once per
-// device; the host-side symbol itself is not a device address).
+// Device address of g_noalloc_scratch on the current device (the host-side
+// symbol itself is not a device address), looked up on the first call in each
+// context of the device: once per device unless the device is reset.
 fa_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= fa::kMaxDevices) return FA_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (g_noalloc_ptr[dev] == nullptr || g_noalloc_ctx[dev] != fa::current_ctx_id()) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = fa::current_ctx_id();
   }
   *out = g_noalloc_ptr[dev];
   return FA_OK;

@@ -346,7 +346,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
         const int kv0 = j * 128;
-        if (kv0 + 128 > lim_min) {          // diagonal or tail block: mask keys >= lim
+        const bool masked = kv0 + 128 > lim_min;   // uniform over the warpgroup
+        if (masked) {                       // diagonal or tail block: mask keys >= lim
           const int cut = lim - kv0;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -382,19 +383,25 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float2 negm = make_float2(-m_use * c2, -m_use * c2);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         uint32_t pr[64];
+        // A block with masked keys takes every exponential on the special-function
+        // unit, whose 2^-inf is exactly 0, so masked keys add exactly nothing to l
+        // and P; those blocks are one per row block, the rest keep the FMA share.
+        auto exp_pack = [&](auto all_mufu) {
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2v, negm);
-          float2 p;
-          if ((0x92u >> ((c >> 1) & 7)) & 1u) {
-            p = ex2_poly2(x);
-          } else {
-            p.x = ex2_approx(x.x);
-            p.y = ex2_approx(x.y);
+          for (int c = 0; c < 128; c += 2) {
+            const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2v, negm);
+            float2 p;
+            if (!decltype(all_mufu)::value && ((0x92u >> ((c >> 1) & 7)) & 1u)) {
+              p = ex2_poly2(x);
+            } else {
+              p.x = ex2_approx(x.x);
+              p.y = ex2_approx(x.y);
+            }
+            if ((c >> 1) & 1) acc1 = fadd2(acc1, p); else acc0 = fadd2(acc0, p);
+            pr[c >> 1] = pack_bf16x2(p.x, p.y);
           }
-          if ((c >> 1) & 1) acc1 = fadd2(acc1, p); else acc0 = fadd2(acc0, p);
-          pr[c >> 1] = pack_bf16x2(p.x, p.y);
-        }
+        };
+        if (masked) exp_pack(BoolTag<true>{}); else exp_pack(BoolTag<false>{});
         const float2 acc = fadd2(acc0, acc1);
         l += acc.x + acc.y;
         tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pr));

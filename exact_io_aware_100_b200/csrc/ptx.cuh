@@ -378,6 +378,12 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
+// Compile-time flag for generic lambdas (a loop body instantiated twice).
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
+
 // Exact widening of two packed bf16 values (low half first) to fp32.
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));

@@ -84,7 +84,7 @@ WORKLOADS = {
     "prefill_gqa": Workload("prefill_gqa", 2, 32, 8192, 128, True, "bf16", 2.0, 1006, False, 8),
     # decoding one token per sequence against an 8192-key cache, 32 query heads over 8 key/value heads
     "decode": Workload("decode", 16, 32, 8192, 128, True, "bf16", 1.0, 1007, False, 8, 1),
-    # head dim 256 (forward): 16 heads of 8192 rows, causal
+    # head dim 256: 16 heads of 8192 rows, causal
     "prefill_d256": Workload("prefill_d256", 2, 16, 8192, 256, True, "bf16", 1.0, 1009),
     # a packed batch of 16 sequences of mixed lengths (up to 8192), causal
     "varlen": Workload("varlen", 16, 32, 8192, 128, True, "bf16", 1.0, 1008, varlen=True),

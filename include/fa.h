@@ -31,12 +31,14 @@
  *    anything is launched.  A kernel whose internal wait gives up (a bug, or a
  *    device that stopped making progress) sets a device status word that
  *    fa_get_device_status() reports; outputs are then undefined.
- *  - Supported: d in {64, 128} for the forward and the backward; d == 256 for
- *    the bf16 forward only (fa_fwd, fa_fwd_gqa, fa_fwd_general: one 128-row
- *    query tile per CTA, after the nearauto.com FlashAttention-2 digest's
- *    "head dimensions up to 256"); fa_decode takes d in {64, 128, 256} (the
- *    split-key kernel for d == 128); 1 <= N <= 2^24; B*H*N*d < 2^31
- *    elements per tensor for the square calls.
+ *  - Supported: d in {64, 128, 256} for the bf16 forward and backward (head
+ *    dimensions up to 256: the nearauto.com FlashAttention-2 digest, section
+ *    "新機能: 最大256のヘッドディメンション、マルチクエリアテンション"); the float32
+ *    forward (fa_fwd_ex) takes d in {64, 128}; fa_decode takes d in
+ *    {64, 128, 256} (the split-key kernel for d == 128); 1 <= N <= 2^24;
+ *    B*H*N*d < 2^31 elements per tensor for the square calls.
+ *  - scale must be finite and positive (FA_ERR_INVALID otherwise): the
+ *    kernels take each row's largest unscaled score as the softmax reference.
  */
 #ifndef FA_H
 #define FA_H
@@ -50,7 +52,7 @@ extern "C" {
 
 typedef enum {
   FA_OK = 0,
-  FA_ERR_INVALID = 1,      /* bad sizes (B, H, N < 1, N too large, non-finite scale),
+  FA_ERR_INVALID = 1,      /* bad sizes (B, H, N < 1, N too large), scale not finite and > 0,
                               or (device status) inconsistent packed sequence offsets */
   FA_ERR_UNSUPPORTED = 2,  /* d or dtype not supported by this call                 */
   FA_ERR_ALIGN = 3,        /* null or not 16-byte aligned pointer                     */
@@ -91,7 +93,7 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
 size_t fa_fwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype);
 
 /*
- * Backward, bf16, d in {64, 128}.  Inputs q, k, v, o, dO: [B,H,N,d] bf16; lse from the
+ * Backward, bf16, d in {64, 128, 256}.  Inputs q, k, v, o, dO: [B,H,N,d] bf16; lse from the
  * forward: [B,H,N] float.  Outputs dq, dk, dv: [B,H,N,d] bf16 (written, not
  * accumulated).  workspace: device memory of at least fa_bwd_workspace_size()
  * bytes, 256-byte aligned (holds the fp32 dQ accumulator and per-row D, lse).
@@ -136,7 +138,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *  lse: [B,H,N] float.  dk and dv of a shared head are the sums over its set.
  * Same layout, ownership, alignment, stream and error rules as fa_fwd /
  * fa_bwd, plus FA_ERR_INVALID when H_kv < 1 or H is not a multiple of H_kv.
- * fa_bwd_gqa takes d in {64, 128} and fa_bwd_workspace_size(B, H, N, d) bytes of
+ * fa_bwd_gqa takes d in {64, 128, 256} and fa_bwd_workspace_size(B, H, N, d) bytes of
  * workspace (sized by the query heads).
  */
 fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -174,7 +176,7 @@ typedef struct {
 typedef struct {
   int B;                        /* batch entries (sequences)                                   */
   int H, H_kv;                  /* query heads, key/value heads (H a multiple of H_kv)          */
-  int d;                        /* head dim: 64 or 128                                          */
+  int d;                        /* head dim: 64, 128 or 256                                     */
   int Nq, Nk;                   /* fixed lengths: rows per batch entry; packed: an upper bound
                                    on every sequence's length (sets the grid)                   */
   const int32_t* cu_seqlens_q;  /* packed: DEVICE array of B + 1 row offsets; NULL: fixed lengths */
@@ -200,7 +202,7 @@ fa_status fa_fwd_general(const void* q, const void* k, const void* v, void* o, f
                          const fa_layout* layout, float scale, int causal, fa_stream_t stream);
 
 /*
- * Backward with a general layout (d in {64, 128}): the exact gradients of fa_fwd_general.
+ * Backward with a general layout (d in {64, 128, 256}): the exact gradients of fa_fwd_general.
  * Inputs q, k, v, o, dout (strides layout->q, k, v, o, dout) and lse from the
  * forward (its layout); outputs dq, dk, dv (strides layout->dq, dk, dv),
  * written, not accumulated; dk and dv of a shared head sum over its set.
@@ -255,7 +257,8 @@ size_t fa_decode_workspace_size(int B, int H, int H_kv, int Lq, int Nk, int d);
  * never allocates (no cudaMalloc, no allocating library routine).
  *
  * The first call on a device (with that device current) looks up the array's
- * device address; make that first call before any stream capture.  All calls
+ * device address; make that first call before any stream capture.  After a
+ * device reset the next call looks it up again (it is tied to the context).  All calls
  * on a device share the one array and leave their contents in it: the dQ
  * accumulator is cleared on every call, but two calls that overlap on the GPU
  * (different streams, no ordering between them) race and give wrong results.

@@ -12,5 +12,6 @@ from .attention import (  # noqa: F401
     attention_fwd_varlen,
     attention_bwd_varlen,
     attention_fwd_rows,
+    bwd_operand_rounding_bound,
     softmax_merge,
 )

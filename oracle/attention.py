@@ -80,6 +80,7 @@ __all__ = [
     "attention_bwd_varlen",
     "softmax_merge",
     "attention_fwd_blockwise",
+    "bwd_operand_rounding_bound",
 ]
 
 
@@ -442,3 +443,36 @@ def attention_fwd_blockwise(q, k, v, scale: float, causal: bool,
                 o_out[b, h, rows] = O / L[:, None]
                 lse_out[b, h, rows] = M + np.log(L)
     return o_out, lse_out
+
+
+def bwd_operand_rounding_bound(q, k, v, do, scale: float, causal: bool, unit_roundoff: float = 2.0 ** -8):
+    """Elementwise first-order bound on how far rounding the backward's matrix-product
+    operands moves the gradients (a tolerance term for the parity tests, not part
+    of the attention definition).
+
+    A backward on matrix units rounds P and dS to a narrower format with unit
+    roundoff u (2^-8 for bfloat16) before the products dV = P^T dO, dQ = scale dS K
+    and dK = scale dS^T Q.  If each operand entry moves by at most u times its
+    size, the triangle inequality bounds each output entry's move by
+        dV: u (|P|^T |dO|),   dQ: u scale (|dS| |K|),   dK: u scale (|dS|^T |Q|),
+    with P and dS this oracle's own (the ``attention_bwd`` quantities).  Grouped
+    heads (k, v with H_kv heads, as in ``attention_bwd_gqa``): a shared head's
+    bound is the sum over its uses.  Returns (bq, bk, bv) shaped like q, k, v.
+    """
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    B, H, N, _ = q.shape
+    H_kv = k.shape[1]
+    bq = np.empty_like(q)
+    bk, bv = np.zeros_like(k), np.zeros_like(v)
+    rows = np.arange(N)
+    for b in range(B):
+        for h in range(H):
+            g = _kv_head(h, H, H_kv)
+            s = _scores(q[b, h], k[b, g], scale, rows, causal)
+            p, _ = _softmax_rows(s)
+            dp = do[b, h] @ v[b, g].T
+            ds = np.abs(p * (dp - (p * dp).sum(axis=1, keepdims=True)))
+            bq[b, h] = unit_roundoff * scale * (ds @ np.abs(k[b, g]))
+            bk[b, g] += unit_roundoff * scale * (ds.T @ np.abs(q[b, h]))
+            bv[b, g] += unit_roundoff * (p.T @ np.abs(do[b, h]))
+    return bq, bk, bv

@@ -44,6 +44,27 @@ def assert_close(name, got, ref, max_abs=MAX_ABS, rel_l2=REL_L2, scale_max_abs=F
     return ma, rl
 
 
+def assert_close_bwd(name, got, ref, operand_bound, max_abs=MAX_ABS, rel_l2=REL_L2):
+    """Gradient check with the error terms the arithmetic itself fixes, per element:
+        |got - ref| <= max_abs + 2^-8 |ref| + operand_bound,
+    and the relative-L2 bound unchanged.
+
+    2^-8 |ref|: the bf16 output's own rounding (a correctly rounded bf16 value is
+    within 2^-8 |x| of x; at |x| >= 8 that alone exceeds a 2e-2 absolute bound).
+    operand_bound: the oracle's ``bwd_operand_rounding_bound`` for the same inputs,
+    the most that rounding the products' operands P and dS to bf16 can move the
+    entry.  Used where gradients reach several units (keys scaled x2, grouped
+    heads), where the absolute bound alone is below what bf16 operands allow."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert np.isfinite(got).all(), f"{name}: non-finite values"
+    ma, rl = errors(got, ref)
+    excess = np.abs(got - ref) - (max_abs + 2.0 ** -8 * np.abs(ref) + np.asarray(operand_bound, np.float64))
+    worst = float(excess.max()) if excess.size else -1.0
+    assert worst <= 0 and rl <= rel_l2, f"{name}: max_abs={ma:.3e} rel_l2={rl:.3e} excess={worst:.3e}"
+    return ma, rl
+
+
 def assert_lse(got, ref, tol=LSE_ABS):
     ma = float(np.abs(np.asarray(got, np.float64) - ref).max())
     assert np.isfinite(got).all() and ma <= tol, f"lse: max_abs={ma:.3e}"

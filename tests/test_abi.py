@@ -67,7 +67,12 @@ def test_argument_validation_without_device(lib):
     b = lib.fa_bwd
     args = [P16] * 9
     assert b(*args, 1, 1, 128, 96, 0.125, 1, P16, 1 << 30, None) == 2              # bwd d=96
-    assert b(*args, 1, 1, 128, 256, 0.125, 1, P16, 1 << 30, None) == 2             # bwd d=256 (forward only)
+    assert b(*args, 1, 1, 128, 320, 0.125, 1, P16, 1 << 30, None) == 2             # bwd d=320
+    assert b(*args, 1, 1, 128, 256, 0.125, 1, 16, 1 << 30, None) == 4              # bwd d=256 passes to the workspace check
+    assert b(*args, 1, 1, 128, 128, 0.0, 1, P16, 1 << 30, None) == 1               # scale must be positive
+    assert b(*args, 1, 1, 128, 128, -0.125, 1, P16, 1 << 30, None) == 1
+    assert f(P16, P16, P16, P16, P16, 1, 1, 8, 64, 0.0, 0, None) == 1              # fwd scale 0
+    assert f(P16, P16, P16, P16, P16, 1, 1, 8, 64, -1.0, 1, None) == 1             # fwd negative scale
     assert g(P16, P16, P16, P16, P16, 1, 1, 128, 256, 0.125, 0, 1, P16, 1 << 30, None) == 2   # fp32 at d=256
     assert b(*args, 1, 1, 128, 128, 0.125, 1, None, 0, None) == 4                  # no workspace
     need = lib.fa_bwd_workspace_size(1, 1, 128, 128)

@@ -62,12 +62,14 @@ def test_backward_head_dim_64(N, causal):
     check_heads(host, dq, dk, dv, range(B * H), H, causal, 1.0 / np.sqrt(d))
 
 
-def test_backward_multi_head_shape_head_dim_64():
-    """The multi-head configuration's sizes (B=4 H=16 N=2048, d = 64) on sampled heads."""
-    B, H, N, d = 4, 16, 2048, 64
-    host, _ = make_case(B, H, N, d, 9400, names=("q", "k", "v", "do"))
-    dq, dk, dv = run_bwd(host, True)
-    check_heads(host, dq, dk, dv, [0, 21, 42, 63], H, True, 1.0 / np.sqrt(d))
+@pytest.mark.parametrize("name", ["multi_head", "multi_head_causal"])
+def test_backward_multi_head_workload_sampled_heads(name):
+    """The multi-head configuration (B=4 H=16 N=2048, d = 64, causal and not) on sampled heads,
+    with the workload's own seeded inputs."""
+    w = inputs.WORKLOADS[name]
+    host = inputs.make_inputs(w, names=("q", "k", "v", "do"))
+    dq, dk, dv = run_bwd(host, w.causal)
+    check_heads(host, dq, dk, dv, [0, 21, 42, 63], w.H, w.causal, w.scale)
 
 
 def test_backward_many_heads_and_sharp_rows():

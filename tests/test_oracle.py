@@ -14,7 +14,8 @@ import pytest
 import torch
 
 from oracle import (attention_bwd, attention_bwd_gqa, attention_fwd, attention_fwd_blockwise,
-                    attention_fwd_decode, attention_fwd_gqa, attention_fwd_rows, softmax_merge)
+                    attention_fwd_decode, attention_fwd_gqa, attention_fwd_rows, bwd_operand_rounding_bound,
+                    softmax_merge)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
@@ -246,6 +247,60 @@ def test_gradient_sums():
         dq, dk, dv = attention_bwd(q, k, v, do, 0.3, causal)
         np.testing.assert_allclose(dv.sum(2), do.sum(2), atol=1e-12)
         np.testing.assert_allclose(dk.sum(2), 0.0, atol=1e-12)
+
+
+# --- the operand-rounding bound used as a tolerance term -------------------
+
+def _grads_with_rounded_operands(q, k, v, do, scale, causal, group):
+    """Brute force in torch float64: P and dS rounded to bfloat16 before the three
+    products, everything else exact; a shared key/value head sums its uses."""
+    q, k, v, do = (torch.from_numpy(np.ascontiguousarray(x)) for x in (q, k, v, do))
+    B, H, N, _ = q.shape
+    dq, dk, dv = torch.zeros_like(q), torch.zeros_like(k), torch.zeros_like(v)
+    bf = lambda x: x.to(torch.bfloat16).to(torch.float64)  # noqa: E731
+    mask = torch.triu(torch.ones(N, N, dtype=torch.bool), 1)
+    for b in range(B):
+        for h in range(H):
+            g = h // group
+            s = scale * q[b, h] @ k[b, g].T
+            if causal:
+                s = s.masked_fill(mask, float("-inf"))
+            p = torch.softmax(s, dim=1)
+            dp = do[b, h] @ v[b, g].T
+            ds = p * (dp - (p * dp).sum(1, keepdim=True))
+            dv[b, g] += bf(p).T @ do[b, h]
+            dq[b, h] = scale * bf(ds) @ k[b, g]
+            dk[b, g] += scale * bf(ds).T @ q[b, h]
+    return dq.numpy(), dk.numpy(), dv.numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("H,H_kv", [(2, 2), (4, 2)])
+def test_operand_rounding_bound_holds_by_brute_force(causal, H, H_kv):
+    """Rounding P and dS to bfloat16 moves every gradient entry by no more than the bound
+    (u = 2^-8), and the bound is tight enough to mean something: for each of dQ, dK, dV the
+    largest move reaches 40 % of it (a bound missing the scale factor would not)."""
+    B, N, d, scale = 1, 40, 8, 0.35
+    q, do = _rand((B, H, N, d), 91), _rand((B, H, N, d), 92)
+    k, v = _rand((B, H_kv, N, d), 93, 4.0), _rand((B, H_kv, N, d), 94)
+    exact = attention_bwd_gqa(q, k, v, do, scale, causal)
+    rounded = _grads_with_rounded_operands(q, k, v, do, scale, causal, H // H_kv)
+    bounds = bwd_operand_rounding_bound(q, k, v, do, scale, causal)
+    for e, r, bnd in zip(exact, rounded, bounds):
+        move = np.abs(r - e)
+        assert (move <= bnd + 1e-12).all(), float((move - bnd).max())
+        worst = float((move / np.maximum(bnd, 1e-300)).max())
+        assert worst > 0.4, worst
+
+
+def test_operand_rounding_bound_scales_with_u_and_vanishes_for_exact_operands():
+    q, k, v, do = (_rand((1, 1, 20, 4), 95 + i) for i in range(4))
+    b1 = bwd_operand_rounding_bound(q, k, v, do, 0.5, True)
+    b2 = bwd_operand_rounding_bound(q, k, v, do, 0.5, True, unit_roundoff=2.0 ** -9)
+    for x, y in zip(b1, b2):
+        np.testing.assert_allclose(x, 2 * y, rtol=1e-14)
+        assert (x >= 0).all()
+    assert all((x == 0).all() for x in bwd_operand_rounding_bound(q, k, v, do, 0.5, True, unit_roundoff=0.0))
 
 
 # --- grouped-query attention ---------------------------------------------
