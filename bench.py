@@ -42,6 +42,7 @@ MUFU_SHARE_OF_EXP = 5 / 8    # both kernels evaluate three of every eight exp2 p
 KERNEL_SOURCES = ["exact_io_aware_100_b200/csrc/ptx.cuh", "exact_io_aware_100_b200/csrc/layout.cuh",
                   "exact_io_aware_100_b200/csrc/fwd_kernel.cuh", "exact_io_aware_100_b200/csrc/bwd_kernel.cuh",
                   "exact_io_aware_100_b200/csrc/fwd256_kernel.cuh", "exact_io_aware_100_b200/csrc/bwd256_kernel.cuh",
+                  "exact_io_aware_100_b200/csrc/fwd64_kernel.cuh",
                   "exact_io_aware_100_b200/csrc/fa_api.cu"]
 
 

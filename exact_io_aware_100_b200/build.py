@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfa.so")
 SOURCES = ["fa_api.cu"]
-DEPS = ["fa_api.cu", "fwd_kernel.cuh", "bwd_kernel.cuh", "bwd256_kernel.cuh", "decode_kernel.cuh", "fwd256_kernel.cuh", "layout.cuh", "ptx.cuh"]
+DEPS = ["fa_api.cu", "fwd_kernel.cuh", "bwd_kernel.cuh", "bwd256_kernel.cuh", "decode_kernel.cuh", "decode_warp_kernel.cuh", "fwd64_kernel.cuh", "fwd256_kernel.cuh", "layout.cuh", "ptx.cuh"]
 
 
 def nvcc_path() -> str:

@@ -220,8 +220,11 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs this loop (its operands are warp-uniform) and one
+    // elected lane issues each MMA and commit: measured faster than a loop run
+    // by lane 0 alone.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 112;");
-    if (lane == 0) {
+    {
       // K-major operands advance 32 B per K step inside a 128-byte row and switch
       // region every four steps; MN-major operands advance 16 rows (2 KB).
       const uint64_t dK_k = sdesc_sw128(sK, 16, 1024), dV_k = sdesc_sw128(sV, 16, 1024);
@@ -240,58 +243,58 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       auto issue_sd = [&](uint32_t d_tmem, uint64_t a, uint64_t bq, int half, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ss(d_tmem, a + kv_step(half, kk), bq + qh_step(kk), C::IDESC_SD, (acc || kk > 0) ? 1u : 0u);
+          umma_ss_elect(d_tmem, a + kv_step(half, kk), bq + qh_step(kk), C::IDESC_SD, (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(b_kv_full, 0, ctl);
+      bool ok = mbar_wait_warp(b_kv_full, 0, ctl);
       for (int it = 0; it < n_iter && ok; ++it) {
         const uint32_t ph = static_cast<uint32_t>(it) & 1u, pp = ph ^ 1u;
         // ---- S^T = K Q^T: the early (not owned) half of d first
-        if (it > 0 && !mbar_wait(b_s_free, pp, ctl)) { ok = false; break; }
-        if (!mbar_wait(b_qoth_full, ph, ctl)) { ok = false; break; }
+        if (it > 0 && !mbar_wait_warp(b_s_free, pp, ctl)) { ok = false; break; }
+        if (!mbar_wait_warp(b_qoth_full, ph, ctl)) { ok = false; break; }
         tc_fence_after();
         issue_sd(tmem + C::T_S, dK_k, dQoth_k, oth, false);
-        umma_commit(b_qoth_empty);
-        if (!mbar_wait(b_qown_full, ph, ctl)) { ok = false; break; }
+        umma_commit_elect(b_qoth_empty);
+        if (!mbar_wait_warp(b_qown_full, ph, ctl)) { ok = false; break; }
         tc_fence_after();
         issue_sd(tmem + C::T_S, dK_k, dQown_k, own, true);
-        umma_commit(b_s_full);
+        umma_commit_elect(b_s_full);
         // ---- dP^T = V dO^T
-        if (it > 0 && !mbar_wait(b_dp_free, pp, ctl)) { ok = false; break; }
-        if (!mbar_wait(b_dooth_full, ph, ctl)) { ok = false; break; }
+        if (it > 0 && !mbar_wait_warp(b_dp_free, pp, ctl)) { ok = false; break; }
+        if (!mbar_wait_warp(b_dooth_full, ph, ctl)) { ok = false; break; }
         tc_fence_after();
         issue_sd(tmem + C::T_DP, dV_k, dDOoth_k, oth, false);
-        umma_commit(b_dooth_empty);
-        if (!mbar_wait(b_doown_full, ph, ctl)) { ok = false; break; }
+        umma_commit_elect(b_dooth_empty);
+        if (!mbar_wait_warp(b_doown_full, ph, ctl)) { ok = false; break; }
         tc_fence_after();
         issue_sd(tmem + C::T_DP, dV_k, dDOown_k, own, true);
-        umma_commit(b_dp_full);
+        umma_commit_elect(b_dp_full);
         // ---- dV_c += P^T dO_c (A = P^T in TMEM, 8 packed columns per 16 queries)
-        if (!mbar_wait(b_p_ready, ph, ctl)) { ok = false; break; }
+        if (!mbar_wait_warp(b_p_ready, ph, ctl)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BM / 16; ++kk)
-          umma_ts(tmem + C::T_DV, tmem + C::T_P + 8 * kk, dDOown_mn + mn_step(kk), C::IDESC_KV,
+          umma_ts_elect(tmem + C::T_DV, tmem + C::T_P + 8 * kk, dDOown_mn + mn_step(kk), C::IDESC_KV,
                   (it > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(b_doown_empty);
-        umma_commit(b_p_free);
+        umma_commit_elect(b_doown_empty);
+        umma_commit_elect(b_p_free);
         // ---- dK_c += dS^T Q_c, then dQ^T_c = K_c^T dS^T
-        if (!mbar_wait(b_ds_ready, ph, ctl)) { ok = false; break; }
+        if (!mbar_wait_warp(b_ds_ready, ph, ctl)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BM / 16; ++kk)
-          umma_ss(tmem + C::T_DK, dDS_k + static_cast<uint64_t>((kk * 32) >> 4), dQown_mn + mn_step(kk), C::IDESC_KV,
+          umma_ss_elect(tmem + C::T_DK, dDS_k + static_cast<uint64_t>((kk * 32) >> 4), dQown_mn + mn_step(kk), C::IDESC_KV,
                   (it > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(b_qown_empty);
-        if (it > 0 && !mbar_wait(b_dq_free, pp, ctl)) { ok = false; break; }
+        umma_commit_elect(b_qown_empty);
+        if (it > 0 && !mbar_wait_warp(b_dq_free, pp, ctl)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          umma_ss(tmem + C::T_DQ, dKown_mn + mn_step(kk), dDS_mn + mn_step(kk), C::IDESC_Q, kk > 0 ? 1u : 0u);
-        umma_commit(b_dq_full);
-        umma_commit(b_ds_free);
+          umma_ss_elect(tmem + C::T_DQ, dKown_mn + mn_step(kk), dDS_mn + mn_step(kk), C::IDESC_Q, kk > 0 ? 1u : 0u);
+        umma_commit_elect(b_dq_full);
+        umma_commit_elect(b_ds_free);
       }
-      if (ok) umma_commit(b_dkv_done);
-      umma_commit(smem_u32(drain_bar));
+      if (ok) umma_commit_elect(b_dkv_done);
+      umma_commit_elect(smem_u32(drain_bar));
       mbar_wait_quiet(smem_u32(drain_bar), 0, 200000000ull);
     }
   } else if (warp < 8) {

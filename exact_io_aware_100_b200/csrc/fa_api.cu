@@ -8,11 +8,14 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "bwd256_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "decode_kernel.cuh"
+#include "decode_warp_kernel.cuh"
 #include "fwd256_kernel.cuh"
+#include "fwd64_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace fa {
@@ -32,7 +35,7 @@ struct DevState {
   bool fwd_attr[2][2] = {}, bwd_attr[2][2] = {};   // [d == 128][packed]: attributes set, registers checked
   bool bwd256_attr[2] = {};                        // [packed]
   bool fwd256_attr[2] = {};                        // [packed]
-  bool dec_attr = false;
+  bool dec_attr = false, decw_attr = false;
 };
 DevState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -287,12 +290,20 @@ bool launch_regs_are(const void* fn, int regs) {
   return cudaFuncGetAttributes(&fa_attr, fn) == cudaSuccess && fa_attr.numRegs == regs;
 }
 
+// The forward kernel for head dim D: fa_fwd64_kernel (its own product order) at
+// D = 64, fa_fwd_kernel otherwise.
+template <int D, bool PACKED>
+constexpr auto fwd_kernel_for() {
+  if constexpr (D == 64) return fa_fwd64_kernel<PACKED>;
+  else return fa_fwd_kernel<D, PACKED>;
+}
+
 template <int D>
 fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, void* o, float* lse,
                      const fa_layout& L, float scale, int causal, int o_f32, cudaStream_t stream) {
-  using C = FwdCfg<D>;
+  using C = std::conditional_t<D == 64, Fwd64Cfg, FwdCfg<D>>;
   const bool pk = packed(L);
-  auto kern = pk ? fa_fwd_kernel<D, true> : fa_fwd_kernel<D, false>;
+  auto kern = pk ? fwd_kernel_for<D, true>() : fwd_kernel_for<D, false>();
   bool& attr = ds->fwd_attr[D == 128][pk];
   if (!attr) {
     if (!launch_regs_are(reinterpret_cast<const void*>(kern), C::LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
@@ -790,9 +801,17 @@ fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float*
       return FA_ERR_CUDA;
     ds->dec_attr = true;
   }
+  // at most four query rows per key/value head: the warp-independent kernel (16-key tiles)
+  const bool warp_tiles = (H / H_kv) * Lq <= DecWCfg::R;
+  if (warp_tiles && !ds->decw_attr) {
+    if (cudaFuncSetAttribute(fa_decode_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecWCfg::SMEM_BYTES) != cudaSuccess)
+      return FA_ERR_CUDA;
+    ds->decw_attr = true;
+  }
   CUtensorMap tk, tv;
-  if (!make_map(&tk, k, d, Nk, B * H_kv, DecCfg::KT) || !make_map(&tv, v, d, Nk, B * H_kv, DecCfg::KT))
-    return FA_ERR_CUDA;
+  const int kt = warp_tiles ? DecWCfg::KT : DecCfg::KT;
+  if (!make_map(&tk, k, d, Nk, B * H_kv, kt) || !make_map(&tv, v, d, Nk, B * H_kv, kt)) return FA_ERR_CUDA;
   DecArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -815,7 +834,9 @@ fa_status fa_decode(const void* q, const void* k, const void* v, void* o, float*
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const dim3 grid(a.n_splits, a.bh_kv);
   const int rows_per_set = a.group * Lq;
-  if (rows_per_set <= 4)
+  if (warp_tiles)
+    fa_decode_warp_kernel<<<grid, DecWCfg::THREADS, DecWCfg::SMEM_BYTES, s>>>(tk, tv, a);
+  else if (rows_per_set <= 4)
     fa_decode_kernel<4><<<grid, DecCfg::THREADS, DecCfg::SMEM_BYTES, s>>>(tk, tv, a);
   else if (rows_per_set <= 8)
     fa_decode_kernel<8><<<grid, DecCfg::THREADS, DecCfg::SMEM_BYTES, s>>>(tk, tv, a);

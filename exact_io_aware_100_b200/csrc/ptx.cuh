@@ -185,6 +185,36 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
                ::"r"(bar) : "memory");
 }
 
+// The same three, issued by one elected lane of a converged warp: every lane
+// computes the (warp-uniform) operands and reaches the instruction, and only
+// the leader lane (the lowest active one, the same lane every time) issues it,
+// so commits track the MMAs that lane issued.
+__device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void umma_commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+      ::"r"(bar) : "memory");
+}
+
 // Shared memory matrix descriptor, 128-byte swizzle, sm_100 version field = 1.
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo_bytes,
                                                 uint32_t sbo_bytes) {
@@ -377,12 +407,6 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
   return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
-
-// Compile-time flag for generic lambdas (a loop body instantiated twice).
-template <bool B>
-struct BoolTag {
-  static constexpr bool value = B;
-};
 
 // Exact widening of two packed bf16 values (low half first) to fp32.
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {

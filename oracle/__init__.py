@@ -2,6 +2,7 @@
 from .attention import (  # noqa: F401
     as_f64,
     attention_bwd,
+    attention_bwd_sampled,
     attention_bwd_gqa,
     attention_fwd,
     attention_fwd_gqa,

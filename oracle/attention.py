@@ -81,6 +81,7 @@ __all__ = [
     "softmax_merge",
     "attention_fwd_blockwise",
     "bwd_operand_rounding_bound",
+    "attention_bwd_sampled",
 ]
 
 
@@ -183,6 +184,38 @@ def attention_bwd(q, k, v, do, scale: float, causal: bool):
             dq[b, h] = scale * (ds @ k[b, h])
             dk[b, h] = scale * (ds.T @ q[b, h])
     return dq, dk, dv
+
+
+def attention_bwd_sampled(q, k, v, do, rows, keys, scale: float, causal: bool, panel_rows: int = 2048):
+    """Selected entries of the exact gradients of ONE head, for sequences too long to
+    hold S: dQ at query rows ``rows`` and dK, dV at key rows ``keys``.
+
+    Same definition as ``attention_bwd`` ([P5] "تکنیک 2: محاسبه مجدد", read as the
+    exact derivative): with P_ij = exp(scale q_i.k_j - lse_i) (masked entries 0),
+    dP_ij = dO_i.v_j and D_i = sum_c dO_ic O_ic,
+        dQ_i = scale sum_j P_ij (dP_ij - D_i) k_j,
+        dV_j = sum_i P_ij dO_i,      dK_j = scale sum_i P_ij (dP_ij - D_i) q_i.
+    lse and O of every row come from ``attention_fwd`` (complete rows, in panels);
+    each requested dQ row then takes its complete row of P, and each requested key
+    its complete column.  q, k, v, do are [N, d]; returns (dq [len(rows), d],
+    dk [len(keys), d], dv [len(keys), d]) in float64.
+    """
+    q, k, v, do = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    N = q.shape[0]
+    o, lse = attention_fwd(q[None, None], k[None, None], v[None, None], scale, causal, panel_rows)
+    o, lse = o[0, 0], lse[0, 0]
+    dd = (do * o).sum(axis=1)
+    rows = np.asarray(rows, dtype=np.int64)
+    keys = np.asarray(keys, dtype=np.int64)
+    s = _scores(q[rows], k, scale, rows, causal)                      # complete rows
+    p = np.exp(s - lse[rows, None])
+    dq = scale * ((p * (do[rows] @ v.T - dd[rows, None])) @ k)
+    st = scale * (q @ k[keys].T)                                      # complete columns
+    if causal:
+        st = np.where(keys[None, :] > np.arange(N)[:, None], -np.inf, st)
+    pt = np.exp(st - lse[:, None])
+    dst = pt * (do @ v[keys].T - dd[:, None])
+    return dq, scale * (dst.T @ q), pt.T @ do
 
 
 def _kv_head(h: int, H: int, H_kv: int) -> int:

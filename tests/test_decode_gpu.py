@@ -27,6 +27,11 @@ def _case(B, H, H_kv, Lq, Nk, seed, k_scale=1.0):
     (1, 2, 2, 16, 2049, True),      # 16 tokens per head (causal bottom-right inside the last tile)
     (3, 6, 3, 8, 5000, False),
     (1, 16, 2, 2, 65536, True),     # long cache: many splits
+    (4, 8, 4, 1, 8192, False),      # two rows per key/value head (warp-tiled kernel)
+    (1, 4, 1, 1, 100, True),        # four rows, cache shorter than one split's first tiles
+    (2, 4, 2, 2, 333, True),        # two query heads x two positions (causal inside the last tile)
+    (1, 3, 1, 1, 17, True),         # three rows, one partial tile
+    (2, 2, 2, 1, 1, True),          # a single cached key
 ])
 def test_decode_matches_oracle(B, H, H_kv, Lq, Nk, causal):
     import torch
@@ -88,5 +93,23 @@ def test_decode_other_shapes_match_oracle(B, H, H_kv, Lq, Nk, d, causal):
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == fa.FA_OK
     ro, rl = attention_fwd_decode(f64["q"], f64["k"], f64["v"], 1.0 / np.sqrt(d), causal)
+    assert_close("O", to_f64(o), ro)
+    assert_lse(to_f64(lse), rl)
+
+
+def test_decode_workload_full_size():
+    """The benchmarked decode workload: 16 sequences, 32 query heads over 8 key/value heads, one
+    new token against 8192 cached keys, every query head checked."""
+    import torch
+    import exact_io_aware_100_b200 as fa
+    w = inputs.WORKLOADS["decode"]
+    shapes = {"q": (w.B, w.H, w.lq, w.d), "k": (w.B, w.kv_heads, w.N, w.d), "v": (w.B, w.kv_heads, w.N, w.d)}
+    host = {n: inputs.make_tensor(w.seed, n, shp) for n, shp in shapes.items()}
+    q, k, v = (to_device(host[n], "bf16") for n in ("q", "k", "v"))
+    o, lse = fa.decode(q, k, v, w.causal)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == fa.FA_OK
+    f64 = {n: inputs.to_f64(x, "bf16") for n, x in host.items()}
+    ro, rl = attention_fwd_decode(f64["q"], f64["k"], f64["v"], w.scale, w.causal)
     assert_close("O", to_f64(o), ro)
     assert_lse(to_f64(lse), rl)

@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (attention_bwd, attention_bwd_gqa, attention_fwd, attention_fwd_blockwise,
+from oracle import (attention_bwd, attention_bwd_gqa, attention_bwd_sampled, attention_fwd, attention_fwd_blockwise,
                     attention_fwd_decode, attention_fwd_gqa, attention_fwd_rows, bwd_operand_rounding_bound,
                     softmax_merge)
 
@@ -247,6 +247,42 @@ def test_gradient_sums():
         dq, dk, dv = attention_bwd(q, k, v, do, 0.3, causal)
         np.testing.assert_allclose(dv.sum(2), do.sum(2), atol=1e-12)
         np.testing.assert_allclose(dk.sum(2), 0.0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_gradients_match_the_whole_gradients(causal):
+    """attention_bwd_sampled equals attention_bwd on the selected rows and keys (panels smaller
+    than N, so the forward it relies on runs in several panels)."""
+    N, d, scale = 300, 16, 0.25
+    q, k, v, do = (_rand((1, 1, N, d), 70 + i, 2.0 if i == 1 else 1.0) for i in range(4))
+    dq, dk, dv = attention_bwd(q, k, v, do, scale, causal)
+    rows, keys = np.array([0, 1, 77, 150, 299]), np.array([0, 5, 150, 298, 299])
+    sq, sk, sv = attention_bwd_sampled(q[0, 0], k[0, 0], v[0, 0], do[0, 0], rows, keys, scale, causal, panel_rows=64)
+    np.testing.assert_allclose(sq, dq[0, 0, rows], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(sk, dk[0, 0, keys], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(sv, dv[0, 0, keys], rtol=1e-11, atol=1e-13)
+
+
+def test_sampled_gradients_by_central_differences():
+    """Independent of attention_bwd: the sampled entries against central differences of the loss."""
+    N, d, scale, h = 7, 3, 0.7, 1e-6
+    q, k, v, do = (_rand((N, d), 74 + i) for i in range(4))
+    rows, keys = np.array([0, 4, 6]), np.array([1, 6])
+    sq, sk, sv = attention_bwd_sampled(q, k, v, do, rows, keys, scale, True)
+
+    def loss(qq, kk, vv):
+        o, _ = attention_fwd(qq[None, None], kk[None, None], vv[None, None], scale, True)
+        return float((o[0, 0] * do).sum())
+
+    for which, idx_rows, got in ((0, rows, sq), (1, keys, sk), (2, keys, sv)):
+        for a, r in enumerate(idx_rows):
+            for c in range(d):
+                args = [q.copy(), k.copy(), v.copy()]
+                args[which][r, c] += h
+                lp = loss(*args)
+                args[which][r, c] -= 2 * h
+                fd = (lp - loss(*args)) / (2 * h)
+                assert abs(fd - got[a, c]) <= 1e-6 * max(1.0, abs(fd)), (which, r, c, fd, got[a, c])
 
 
 # --- the operand-rounding bound used as a tolerance term -------------------

@@ -17,8 +17,8 @@ import numpy as np
 import pytest
 
 from exact_io_aware_100_b200 import inputs
-from oracle import (attention_bwd, attention_bwd_gqa, attention_bwd_varlen, attention_fwd_rows,
-                    attention_fwd_varlen, bwd_operand_rounding_bound)
+from oracle import (attention_bwd, attention_bwd_gqa, attention_bwd_sampled, attention_bwd_varlen,
+                    attention_fwd_rows, attention_fwd_varlen, bwd_operand_rounding_bound)
 from tests.helpers import assert_close, assert_close_bwd, assert_lse, to_device, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -173,3 +173,27 @@ def test_varlen_full_size_sampled_sequences():
     for name in ("dq", "dk", "dv"):
         assert_close(name, np.concatenate(got[name]), np.concatenate(ref[name]))
     assert np.isfinite(o64).all() and np.isfinite(lse64).all()
+
+
+def test_long_context_backward_sampled():
+    """B=1 H=16 N=65536 d=128, causal (the long-context configuration; the benchmark times its
+    forward and backward): dQ on 128 sampled query rows and dK, dV on 128 sampled keys of one
+    head, each against the oracle's complete row or column (the oracle's forward runs the whole
+    head in panels for lse and O)."""
+    import exact_io_aware_100_b200 as fa
+    w = inputs.WORKLOADS["long_context"]
+    host = inputs.make_inputs(w, names=("q", "k", "v", "do"))
+    t = _bf16(host)
+    o, lse = fa.forward(t["q"], t["k"], t["v"], w.causal)
+    dq, dk, dv = fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], w.causal)
+    _status_ok()
+    h = 11
+    rows = inputs.sample_rows(w.seed + 5, w.N, 128)
+    keys = inputs.sample_rows(w.seed + 6, w.N, 128)
+    f = {n: inputs.to_f64(host[n][0, h], "bf16") for n in ("q", "k", "v", "do")}
+    rq, rk, rv = attention_bwd_sampled(f["q"], f["k"], f["v"], f["do"], rows, keys, w.scale, w.causal)
+    assert_close("dq(sampled rows)", to_f64(dq[0, h, rows]), rq)
+    assert_close("dk(sampled keys)", to_f64(dk[0, h, keys]), rk)
+    assert_close("dv(sampled keys)", to_f64(dv[0, h, keys]), rv)
+    for x in (dq, dk, dv):
+        assert np.isfinite(to_f64(x)).all()
