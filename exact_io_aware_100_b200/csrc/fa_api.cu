@@ -290,20 +290,29 @@ bool launch_regs_are(const void* fn, int regs) {
   return cudaFuncGetAttributes(&fa_attr, fn) == cudaSuccess && fa_attr.numRegs == regs;
 }
 
-// The forward kernel for head dim D: fa_fwd64_kernel (its own product order) at
-// D = 64, fa_fwd_kernel otherwise.
-template <int D, bool PACKED>
-constexpr auto fwd_kernel_for() {
-  if constexpr (D == 64) return fa_fwd64_kernel<PACKED>;
-  else return fa_fwd_kernel<D, PACKED>;
-}
+// The forward kernel a head dim uses: at d = 64 the one with separate P buffers
+// (next scores computed during the softmax), at d = 128 the ping-pong kernel.
+template <int D>
+struct FwdPlan;
+template <>
+struct FwdPlan<64> {
+  using C = FwdSpCfg<64, 128>;
+  template <bool PACKED>
+  static constexpr auto kernel() { return fa_fwd_sp_kernel<64, 128, PACKED>; }
+};
+template <>
+struct FwdPlan<128> {
+  using C = FwdCfg<128>;
+  template <bool PACKED>
+  static constexpr auto kernel() { return fa_fwd_kernel<128, PACKED>; }
+};
 
 template <int D>
 fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, void* o, float* lse,
                      const fa_layout& L, float scale, int causal, int o_f32, cudaStream_t stream) {
-  using C = std::conditional_t<D == 64, Fwd64Cfg, FwdCfg<D>>;
+  using C = typename FwdPlan<D>::C;
   const bool pk = packed(L);
-  auto kern = pk ? fwd_kernel_for<D, true>() : fwd_kernel_for<D, false>();
+  auto kern = pk ? FwdPlan<D>::template kernel<true>() : FwdPlan<D>::template kernel<false>();
   bool& attr = ds->fwd_attr[D == 128][pk];
   if (!attr) {
     if (!launch_regs_are(reinterpret_cast<const void*>(kern), C::LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
@@ -314,8 +323,8 @@ fa_status launch_fwd(DevState* ds, const void* q, const void* k, const void* v, 
   if (L.Nq == 0 || (packed(L) && L.total_q == 0)) return FA_OK;   // no query row: nothing to write
   CUtensorMap tq, tk, tv;
   const int bq = batches(L);
-  if (!make_map4(&tq, q, D, q_rows(L), L.H, bq, L.q) || !make_map4(&tk, k, D, k_rows(L), L.H_kv, bq, L.k) ||
-      !make_map4(&tv, v, D, k_rows(L), L.H_kv, bq, L.v))
+  if (!make_map4(&tq, q, D, q_rows(L), L.H, bq, L.q) || !make_map4(&tk, k, D, k_rows(L), L.H_kv, bq, L.k, C::BN) ||
+      !make_map4(&tv, v, D, k_rows(L), L.H_kv, bq, L.v, C::BN))
     return FA_ERR_CUDA;
   FwdArgs a;
   a.o = o;

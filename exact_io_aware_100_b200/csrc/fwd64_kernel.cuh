@@ -28,12 +28,14 @@
 
 namespace fa {
 
-struct Fwd64Cfg {
-  static constexpr int D = 64;
+template <int D_, int BN_>
+struct FwdSpCfg {
+  static constexpr int D = D_;
   static constexpr int BM = 128;                  // query rows per softmax warpgroup
-  static constexpr int BN = 128;                  // keys per KV block
-  static constexpr int REGION = 128 * 128;        // one 64-column (128 B) swizzle region of a 128-row tile
-  static constexpr int N_REG = 1;                 // regions per 128-row tile
+  static constexpr int BN = BN_;                  // keys per KV block
+  static constexpr int REGION = 128 * 128;        // one 64-column (128 B) swizzle region of a 128-row Q half
+  static constexpr int KV_REGION = BN * 128;      // one 64-column region of a BN-row K or V block
+  static constexpr int N_REG = D / 64;            // regions per row
   static constexpr int Q_HALF = BM * D * 2;       // bytes of one 128-row Q half
   static constexpr int KV_BYTES = BN * D * 2;     // bytes of one K or V block
   static constexpr int STAGES = 8;
@@ -42,7 +44,8 @@ struct Fwd64Cfg {
   // the eight softmax warps take 224, the other four give theirs down to 56.
   static constexpr int LAUNCH_REGS = 168;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 320, T_P0 = 384, T_P1 = 448;
+  static constexpr uint32_t T_O0 = 0, T_O1 = D, T_S0 = 2 * D, T_S1 = 2 * D + BN, T_P0 = 2 * D + 2 * BN,
+                            T_P1 = 2 * D + 2 * BN + BN / 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_HALF;
   static constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
@@ -52,14 +55,28 @@ struct Fwd64Cfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024; // + alignment slack
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
+  static_assert(T_P1 + BN / 2 <= TMEM_COLS, "tensor memory plan");
+  static_assert(SMEM_BYTES <= 232448, "shared memory plan");
 };
+using Fwd64Cfg = FwdSpCfg<64, 128>;
 
-template <bool PACKED>
-__global__ void __launch_bounds__(Fwd64Cfg::THREADS, 1)
-fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
-  using C = Fwd64Cfg;
-  constexpr int D = C::D;
+// Key blocks of BN keys that tile qt (256 query rows) of sequence s reads.
+template <int BN>
+__host__ __device__ __forceinline__ int fwd_num_kv_bn(const FwdArgs& a, const SeqSpan& s, int qt) {
+  if (qt * 256 >= s.nq) return 0;
+  const int n_all = (s.nk + BN - 1) / BN;
+  if (!a.causal) return n_all;
+  const int last_row = min(qt * 256 + 255, s.nq - 1);
+  const int vis = last_row + (s.nk - s.nq) + 1;       // keys < vis are visible to the last row
+  return vis <= 0 ? 0 : min((vis + BN - 1) / BN, n_all);
+}
+
+template <int D_, int BN_, bool PACKED>
+__global__ void __launch_bounds__(FwdSpCfg<D_, BN_>::THREADS, 1)
+fa_fwd_sp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
+  using C = FwdSpCfg<D_, BN_>;
+  constexpr int D = C::D, BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -125,7 +142,7 @@ fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int b, h, qt;
         fwd_decode_tile(args, t, b, h, qt);
         const SeqSpan sp = seq_span<PACKED>(args.L, b, args.status);
-        const int nkv = fwd_num_kv(args, sp, qt);
+        const int nkv = fwd_num_kv_bn<BN>(args, sp, qt);
         if (nkv == 0) continue;                        // nothing to load for this tile
         const int h_kv = h / args.group;
         if (tile_cnt > 0 && !mbar_wait(b_q_empty, (tile_cnt - 1) & 1, ctl)) { ok = false; break; }
@@ -144,7 +161,7 @@ fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_expect_tx(b_kv_full(s), C::KV_BYTES);
             const CUtensorMap* map = kind ? &tm_v : &tm_k;
             for (int r = 0; r < C::N_REG; ++r)
-              tma_load_4d(sKV + s * C::KV_BYTES + r * C::REGION, map, b_kv_full(s), r * 64, sp.k0 + j * 128, h_kv,
+              tma_load_4d(sKV + s * C::KV_BYTES + r * C::KV_REGION, map, b_kv_full(s), r * 64, sp.k0 + j * BN, h_kv,
                           sp.bc);
             issued |= 1u << s;
             last_parity = (last_parity & ~(1u << s)) | ((round & 1u) << s);
@@ -167,7 +184,7 @@ fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     {
       // descriptor of address a + off == descriptor of a, plus off / 16 (no carry:
       // shared addresses stay below 2^18, the start field holds 14 bits of a / 16)
-      constexpr uint32_t LBO_K = 16, LBO_V = C::REGION, SBO = 1024;
+      constexpr uint32_t LBO_K = 16, LBO_V = C::KV_REGION, SBO = 1024;
       uint32_t kv_it = 0, tile_cnt = 0;
       bool ok = true;
       auto issue_s = [&](uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {   // S = Q K^T
@@ -175,8 +192,9 @@ fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint64_t dk = sdesc_sw128(opaque_u32(k_addr), LBO_K, SBO);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * C::REGION + (kk & 3) * 32) >> 4;
-          umma_ss_elect(d_tmem, dq + off, dk + off, C::IDESC_S, kk > 0);
+          const uint32_t offq = ((kk >> 2) * C::REGION + (kk & 3) * 32) >> 4;
+          const uint32_t offk = ((kk >> 2) * C::KV_REGION + (kk & 3) * 32) >> 4;
+          umma_ss_elect(d_tmem, dq + offq, dk + offk, C::IDESC_S, kk > 0);
         }
       };
       auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, bool acc) {   // O += P V
@@ -192,7 +210,7 @@ fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
         int b, h, qt;
         fwd_decode_tile(args, t, b, h, qt);
-        const int nkv = fwd_num_kv(args, seq_span<PACKED>(args.L, b, args.status), qt);
+        const int nkv = fwd_num_kv_bn<BN>(args, seq_span<PACKED>(args.L, b, args.status), qt);
         if (nkv == 0) continue;
         const uint32_t kv_base = kv_it;
         kv_it += 2u * static_cast<uint32_t>(nkv);
@@ -275,7 +293,7 @@ fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       int b, h, qt;
       fwd_decode_tile(args, t, b, h, qt);
       const SeqSpan sp = seq_span<PACKED>(args.L, b, args.status);
-      const int nkv = fwd_num_kv(args, sp, qt);
+      const int nkv = fwd_num_kv_bn<BN>(args, sp, qt);
       const int row0 = qt * 256 + half * 128;           // rows of the sequence
       const int row = row0 + rloc;
       if (nkv == 0) {                                   // no key visible to any row: O = 0, lse = -inf
@@ -301,36 +319,36 @@ fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!mbar_wait_warp(b_s_full, s_par, ctl)) { ok = false; break; }
         s_par ^= 1;
         tc_fence_after();
-        uint32_t sr[128];
+        uint32_t sr[BN];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < BN / 32; ++c)
           tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+        for (int c = 0; c < BN / 32; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
         tc_fence_before();
         mbar_arrive(b_s_free);                          // the MMA warp may compute S_{j+1} into the buffer
-        float s[128];
+        float s[BN];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-        const int kv0 = j * 128;
-        if (kv0 + 128 > lim_min) {          // diagonal or tail block: mask keys >= lim
+        for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sr[c]);
+        const int kv0 = j * BN;
+        if (kv0 + BN > lim_min) {           // diagonal or tail block: mask keys >= lim
           const int cut = lim - kv0;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < BN; ++c)
             if (c >= cut) s[c] = -INFINITY;
         }
         // row max: four independent chains of 3-input max
         float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-        for (int c = 4; c < 124; c += 8) {
+        for (int c = 4; c < BN - 4; c += 8) {
           mx0 = fmax3(mx0, s[c], s[c + 1]);
           mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
           mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
           mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
         }
-        mx0 = fmax3(mx0, s[124], s[125]);
-        mx1 = fmax3(mx1, s[126], s[127]);
+        mx0 = fmax3(mx0, s[BN - 4], s[BN - 3]);
+        mx1 = fmax3(mx1, s[BN - 2], s[BN - 1]);
         const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
         const float m_new = fmaxf(m_ref, mx);
         const bool need = (m_new - m_ref) * c2 > 8.0f;          // false while the row has seen no key
@@ -349,9 +367,9 @@ fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const float m_use = m_ref == -INFINITY ? 0.0f : m_ref;
         const float2 negm = make_float2(-m_use * c2, -m_use * c2);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-        uint32_t pr[64];
+        uint32_t pr[BN / 2];
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
+        for (int c = 0; c < BN; c += 2) {
           const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2v, negm);
           float2 p;
           if ((0x92u >> ((c >> 1) & 7)) & 1u) {
@@ -370,8 +388,8 @@ fa_fwd64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (blocks > 0 && !mbar_wait_warp(b_pv_done, (blocks - 1) & 1, ctl)) { ok = false; break; }
         ++blocks;
         tc_fence_after();
-        tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(pr));
-        tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(pr + 32));
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) tmem_st32(tP + c * 32, *reinterpret_cast<uint32_t(*)[32]>(pr + c * 32));
         // O rescale (after the scores are dead, to keep register pressure down)
         if (rescale && j > 0) {
           const float2 a2 = make_float2(alpha, alpha);
