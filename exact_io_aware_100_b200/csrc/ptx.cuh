@@ -429,10 +429,5 @@ __device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
 __device__ __forceinline__ void red_add_f32(float* addr, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
-// Four consecutive fp32 atomic adds in one instruction (16-byte aligned address).
-__device__ __forceinline__ void red_add_v4_f32(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 }  // namespace fa
