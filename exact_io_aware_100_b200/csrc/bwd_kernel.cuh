@@ -223,7 +223,7 @@ struct BwdCfg {
   static constexpr int OFF_VEC = OFF_PS + DS_BYTES;   // per Q stage: lse2[BM] then D[BM]
   static constexpr int VEC_BYTES = 2 * BM * 4;
   static constexpr int OFF_BAR = OFF_VEC + 2 * VEC_BYTES;
-  static constexpr int N_BARS = 23;
+  static constexpr int N_BARS = 20;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int USED = OFF_MISC + 16;
   // At most the opt-in maximum per block.  The kernel rounds its base up to 1 KB
@@ -262,27 +262,7 @@ __host__ __device__ __forceinline__ void bwd_decode(const BwdArgs& a, int x, int
   bh = h0 + (r - kb * gh);
 }
 
-// Pair mode: CTAs 2p and 2p + 1 form a cluster over key blocks 2 kp and
-// 2 kp + 1 of one key/value head (pair item p decoded like a work item over
-// ceil(n_kb / 2) key-block pairs).
-__host__ __device__ __forceinline__ void bwd_decode_pair(const BwdArgs& a, int p, int& bh, int& kbp) {
-  const int n_kbp = (a.n_kb + 1) / 2;
-  const int per_group = a.heads_per_group * n_kbp;
-  const int g = p / per_group;
-  const int r = p - g * per_group;
-  const int h0 = g * a.heads_per_group;
-  const int gh = min(a.heads_per_group, a.bh_kv - h0);
-  kbp = r / gh;
-  bh = h0 + (r - kbp * gh);
-}
-
-// PAIR: launched in clusters of two CTAs on neighbouring key blocks.  Both walk
-// the same query blocks (the lower key block first does the one diagonal block
-// the upper one does not see) and split each block's dQ: CTA r adds query rows
-// [64 r, 64 r + 64) to the accumulator, receiving the partner's partial sums of
-// those rows through distributed shared memory, so each accumulator element
-// takes one reduction per key-block pair instead of one per key block.
-template <int D_, bool PACKED, bool PAIR>
+template <int D_, bool PACKED>
 __global__ void __launch_bounds__(BwdCfg<D_>::THREADS, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -291,14 +271,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   constexpr int D = C::D;
   extern __shared__ __align__(16) uint8_t smem_raw[];   // only 16 B promised: the 1 KB rounding below is real
   int bh, kb;                                        // bh: key/value head (b * H_kv + h_kv)
-  const int rank = PAIR ? static_cast<int>(blockIdx.x & 1u) : 0;
-  if constexpr (PAIR) {
-    int kbp;
-    bwd_decode_pair(args, static_cast<int>(blockIdx.x >> 1), bh, kbp);
-    kb = 2 * kbp + rank;
-  } else {
-    bwd_decode(args, static_cast<int>(blockIdx.x), bh, kb);
-  }
+  bwd_decode(args, static_cast<int>(blockIdx.x), bh, kb);
   const int b = bh / args.L.H_kv, h_kv = bh - b * args.L.H_kv;
   const SeqSpan sp = seq_span<PACKED>(args.L, b, args.status);
   const int k0 = kb * C::BN;                         // first key of the block, in the sequence
@@ -306,15 +279,8 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int off = sp.nk - sp.nq;                     // bottom-right causal alignment
   const int n_qb = (sp.nq + C::BM - 1) / C::BM;
   // query blocks that see these keys (every key is seen by the last query row)
-  auto first_qb = [&](int key0) { return args.causal ? max(0, key0 - off) / C::BM : 0; };
-  const int i_begin = first_qb(k0);
+  const int i_begin = args.causal ? max(0, k0 - off) / C::BM : 0;
   const int n_per = max(0, n_qb - i_begin);          // per query head
-  // pair mode: both key blocks of the pair exist (else this CTA works alone);
-  // query blocks >= i_common are walked by both
-  const int k0_pair = (kb ^ 1) * C::BN;
-  const bool paired = PAIR && ((kb | 1) * C::BN < sp.nk);
-  const int i_common = first_qb(max(k0, k0_pair));
-  const int n_per_peer = max(0, n_qb - first_qb(k0_pair));
   const int n_iter = n_per * args.group;             // every query head of the set, one after the other
   if (n_iter == 0) {                                 // no query at all: dK = dV = 0
     const int nk = min(C::BN, sp.nk - k0);
@@ -358,8 +324,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const uint32_t b_yhi_free = bar(17);   // all of Y read out
   const uint32_t b_dkv_done = bar(18);
   const uint32_t b_drain = bar(19);
-  const uint32_t b_px_ok = bar(20);      // pair mode: the partner may push into this block's dO stage
-  auto b_px_full = [&](int h) { return bar(21 + h); };   // pair mode: the partner's 32-row chunk h has landed (tx)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC + 4);
 
@@ -386,9 +350,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     mbar_init(b_yhi_free, C::DRAIN_THREADS);
     mbar_init(b_dkv_done, 1);
     mbar_init(b_drain, 1);
-    mbar_init(b_px_ok, 1);
-    mbar_init(b_px_full(0), 1);
-    mbar_init(b_px_full(1), 1);
     fence_mbar_init();
   }
   if (warp == 12) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -401,7 +362,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (paired) cluster_sync_all();                    // the partner's barriers are initialised
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, args.status, args.wait_limit_ns};
 
@@ -675,17 +635,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // dQ^T_i), and one thread adds it to the accumulator with a bulk reduction:
     // whole lines from one instruction instead of a scalar atomic per element.
     // The stage goes back to the loader once the reductions have read it.
-    // Pair mode, on a block both CTAs walk: the chunks of the partner's half
-    // are stored straight into the partner's dO stage (asynchronous stores to
-    // distributed shared memory, counted in bytes on the partner's barrier), and
-    // the chunks of this CTA's half are added to what the partner stored here
-    // before they are reduced.  Every wait ends in a vote of the four drain
-    // warps, so they leave together.
+    // The wait for each block ends in a vote of the four drain warps, so they
+    // leave together and none is left at a later named barrier.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
     const int dl = (warp - 8) * 32 + lane;
     const bool issuer = dl == 0;
     const uint32_t tY = tmem + (static_cast<uint32_t>((warp - 8) * 32) << 16) + C::T_Y;
-    uint32_t n_common = 0;                           // blocks walked together with the partner so far
     for (int it = 0; it < n_iter; ++it) {
       const int s = it & 1;
       if (!named_bar_and(1, C::DRAIN_THREADS, mbar_wait_warp(b_dq_full, static_cast<uint32_t>(it) & 1, ctl))) break;
@@ -693,20 +648,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const int q0 = q_row0(it);
       const int nq = min(C::BM, sp.nq - q0);
       float* stage = reinterpret_cast<float*>(smem + C::OFF_DO + s * C::TILE);
-      const bool common = paired && q0 / C::BM >= i_common;
-      uint32_t peer_stage = 0;
-      if (common) {
-        // this block's dO stage is free (its readers are done): the partner may push into it,
-        // 32 rows x D fp32 per chunk
-        if (issuer) {
-          mbar_expect_tx(b_px_full(0), C::CHUNK_FLOATS * 4);
-          mbar_expect_tx(b_px_full(1), C::CHUNK_FLOATS * 4);
-          mbar_arrive_cluster(mapa_shared(b_px_ok, static_cast<uint32_t>(rank ^ 1)));
-        }
-        const int it_peer = (it / n_per) * n_per_peer + (q0 / C::BM - first_qb(k0_pair));
-        peer_stage = mapa_shared(sDO(it_peer & 1), static_cast<uint32_t>(rank ^ 1));
-      }
-      bool ok = true;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {      // chunk c: queries 32c .. 32c + 31 of the block
         uint32_t r[32];
@@ -718,41 +659,12 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           mbar_arrive(c == 1 ? b_ylo_free : b_yhi_free);
         }
         const int rows = min(32, nq - 32 * c);       // uniform over the drain warps; later chunks have fewer
-        float* buf = stage + (c & 1) * C::CHUNK_FLOATS;
-        if (common) {
-          if ((c >> 1) != rank) {                    // the partner's rows: store them into its stage
-            if ((c & 1) == 0) {
-              ok = named_bar_and(1, C::DRAIN_THREADS, mbar_wait_cluster_warp(b_px_ok, n_common & 1, ctl));
-              if (!ok) break;
-            }
-            if (dl < D) {
-              const uint32_t dst = peer_stage + static_cast<uint32_t>((c & 1) * C::CHUNK_FLOATS + dl) * 4;
-              const uint32_t pbar = mapa_shared(b_px_full(c & 1), static_cast<uint32_t>(rank ^ 1));
-#pragma unroll
-              for (int j = 0; j < 32; ++j) st_async_f32(dst + j * D * 4, __uint_as_float(r[j]), pbar);
-            }
-          } else {                                   // this CTA's rows: add the partner's sums, then reduce
-            ok = named_bar_and(1, C::DRAIN_THREADS, mbar_wait_cluster_warp(b_px_full(c & 1), n_common & 1, ctl));
-            if (!ok) break;
-            if (dl < D) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) buf[j * D + dl] += __uint_as_float(r[j]);
-            }
-            fence_proxy_async_smem();
-            named_bar_sync(1, C::DRAIN_THREADS);
-            if (issuer && rows > 0) {
-              float* acc = args.dq_acc + (row_index<PACKED>(args.L, sp, q_head(it), q0) + 32 * c) * D;
-              bulk_reduce_add_f32(acc, sDO(s) + (c & 1) * C::CHUNK_FLOATS * 4, static_cast<uint32_t>(rows) * D * 4);
-              bulk_commit();
-            }
-          }
-          continue;
-        }
         if (rows <= 0) continue;
         if (c >= 2) {                                // chunk c - 2 has been read out of this buffer
           if (issuer) bulk_wait_read<1>();
           named_bar_sync(1, C::DRAIN_THREADS);
         }
+        float* buf = stage + (c & 1) * C::CHUNK_FLOATS;
         if (dl < D) {                                // none for the lanes past the head dim (D = 64)
 #pragma unroll
           for (int j = 0; j < 32; ++j) buf[j * D + dl] = __uint_as_float(r[j]);
@@ -765,19 +677,16 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           bulk_commit();
         }
       }
-      if (!ok) break;
       if (issuer) {
         bulk_wait_read<0>();
         mbar_arrive(b_do_empty(s));
       }
-      if (common) ++n_common;
     }
     if (issuer) bulk_wait_all();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (paired) cluster_sync_all();                    // the partner no longer touches this CTA's shared memory
   if (warp == 12) {
     __syncwarp();
     tc_fence_after();

@@ -508,20 +508,15 @@ namespace {
 enum BwdPhase : int { PH_PREPARE = 1, PH_MAIN = 2, PH_FINISH = 4, PH_ALL = 7 };
 
 // First use of a backward main kernel on a device.
-template <int D, bool PACKED, bool PAIR>
-fa_status prepare_bwd_kernel_one() {
-  using C = BwdCfg<D>;
-  if (!launch_regs_are(reinterpret_cast<const void*>(fa_bwd_kernel<D, PACKED, PAIR>), C::LAUNCH_REGS))
-    return FA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(fa_bwd_kernel<D, PACKED, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::SMEM_BYTES) != cudaSuccess)
-    return FA_ERR_CUDA;
-  return FA_OK;
-}
 template <int D, bool PACKED>
 fa_status prepare_bwd_kernel() {
-  const fa_status st = prepare_bwd_kernel_one<D, PACKED, false>();
-  return st != FA_OK ? st : prepare_bwd_kernel_one<D, PACKED, true>();
+  using C = BwdCfg<D>;
+  if (!launch_regs_are(reinterpret_cast<const void*>(fa_bwd_kernel<D, PACKED>), C::LAUNCH_REGS))
+    return FA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(fa_bwd_kernel<D, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
 }
 
 template <bool PACKED>
@@ -534,34 +529,14 @@ fa_status prepare_bwd256_kernel() {
   return FA_OK;
 }
 
-// Pair mode runs the kernel in clusters of two CTAs (neighbouring key blocks).
-template <int D, bool PACKED>
-cudaError_t launch_bwd_main_one(bool pair, unsigned grid, const CUtensorMap& tq, const CUtensorMap& tk,
-                         const CUtensorMap& tv, const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
-  using C = BwdCfg<D>;
-  if (!pair) {
-    fa_bwd_kernel<D, PACKED, false><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
-    return cudaSuccess;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fa_bwd_kernel<D, PACKED, true>, tq, tk, tv, tdo, a);
-}
 template <int D>
-cudaError_t launch_bwd_main(bool pk, bool pair, unsigned grid, const CUtensorMap& tq, const CUtensorMap& tk,
-                            const CUtensorMap& tv, const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
-  return pk ? launch_bwd_main_one<D, true>(pair, grid, tq, tk, tv, tdo, a, stream)
-            : launch_bwd_main_one<D, false>(pair, grid, tq, tk, tv, tdo, a, stream);
+void launch_bwd_main(bool pk, unsigned grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  if (pk)
+    fa_bwd_kernel<D, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  else
+    fa_bwd_kernel<D, false><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
 }
 
 // Validates, fills the kernel arguments, and launches the requested phases.
@@ -651,11 +626,7 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
         !make_map4(&tv, v, d, k_rows(L), L.H_kv, bq, L.v) ||
         !make_map4(&tdo, dout, d, q_rows(L), L.H, bq, L.dout, qbox))
       return FA_ERR_CUDA;
-    // Clusters of two CTAs on neighbouring key blocks can share each query block's dQ reductions
-    // (half the accumulator traffic); not enabled until it measures faster than one CTA per block.
-    const bool pair = false;
-    const long long grid = d == 256 ? 2LL * a.n_kb * a.bh_kv
-                                    : (pair ? 2LL * ((a.n_kb + 1) / 2) : static_cast<long long>(a.n_kb)) * a.bh_kv;
+    const long long grid = static_cast<long long>(a.n_kb) * a.bh_kv * (d == 256 ? 2 : 1);
     if (grid >= (1LL << 31)) return FA_ERR_INVALID;
     if (d == 256) {
       if (pk)
@@ -664,11 +635,10 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
       else
         fa_bwd256_kernel<false><<<static_cast<unsigned>(grid), Bwd256Cfg::THREADS, Bwd256Cfg::SMEM_BYTES, stream>>>(
             tq, tk, tv, tdo, a);
-    } else if ((d == 64 ? launch_bwd_main<64>(pk, pair, static_cast<unsigned>(grid), tq, tk, tv, tdo, a, stream)
-                        : launch_bwd_main<128>(pk, pair, static_cast<unsigned>(grid), tq, tk, tv, tdo, a, stream)) !=
-               cudaSuccess) {
-      return FA_ERR_CUDA;
-    }
+    } else if (d == 64)
+      launch_bwd_main<64>(pk, static_cast<unsigned>(grid), tq, tk, tv, tdo, a, stream);
+    else
+      launch_bwd_main<128>(pk, static_cast<unsigned>(grid), tq, tk, tv, tdo, a, stream);
   }
   if ((phases & PH_FINISH) && a.acc_rows > 0) {
     if (d == 64)

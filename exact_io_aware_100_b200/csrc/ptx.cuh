@@ -92,65 +92,6 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, co
   return __all_sync(0xffffffffu, ok);
 }
 
-// ---------------------------------------------------------------- clusters
-// This CTA's rank in its cluster.
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// The shared::cluster address of `addr` (a shared::cta address of this CTA) in CTA `rank`.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-// Asynchronous store into another CTA's shared memory (shared::cluster
-// addresses); its 4 bytes count against the transaction count of the mbarrier
-// `bar` there, whose phase completes once every expected byte has landed.
-__device__ __forceinline__ void st_async_f32(uint32_t addr, float v, uint32_t bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];"
-               ::"r"(addr), "f"(v), "r"(bar) : "memory");
-}
-// Arrive on an mbarrier of another CTA of the cluster (shared::cluster address),
-// releasing this thread's prior writes at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-  return ok != 0;
-}
-// Bounded wait on a local mbarrier whose arrivals come from another CTA of the
-// cluster (acquire at cluster scope), warp-collective like mbar_wait_warp.
-__device__ __forceinline__ bool mbar_wait_cluster_warp(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
-  bool ok = mbar_try_wait_cluster(bar, parity);
-  if (!ok) {
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-      if (mbar_try_wait_cluster(bar, parity)) { ok = true; break; }
-      if ((it & 63u) == 0u) {
-        if (*ctl.abort) break;
-        if (globaltimer_ns() - t0 > ctl.limit_ns) {
-          atomicOr(ctl.status, DEV_TIMEOUT);
-          *ctl.abort = 1u;
-          break;
-        }
-      }
-    }
-  }
-  return __all_sync(0xffffffffu, ok);
-}
-// Every thread of every CTA of the cluster: arrive, then wait for all.
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 // Teardown wait: bounded, ignores the abort flag, never flags.
 __device__ __forceinline__ bool mbar_wait_quiet(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
