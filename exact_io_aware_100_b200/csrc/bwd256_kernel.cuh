@@ -14,7 +14,7 @@
 //   dP^T = V dO^T       (full d, computed by both CTAs)       TMEM DP
 //   dV_c += P^T dO_c    (A = P^T bf16 in TMEM)                TMEM DV
 //   dK_c += dS^T Q_c    (A = dS^T bf16, shared memory)        TMEM DK
-//   dQ^T_c = K_c^T dS^T (into TMEM DQ, drained with fp32 atomics into dQacc)
+//   dQ^T_c = K_c^T dS^T (into TMEM DQ, added to dQacc by tensor bulk reductions)
 // per block of 64 queries (K, V: 64 KB each, resident; a 64-query block of Q
 // or dO is 32 KB).  Tensor memory: DV 128 | DK 128 | S 64 | DP 64 | DQ 64 |
 // P 32 (of 512) columns.  Q and dO are staged as two 16 KB halves of d each:
@@ -25,7 +25,9 @@
 //
 // Warp roles (448 threads): warps 0-7 compute P and dS (thread = key row,
 // warp w covers the 32 queries 32 (w / 4) .. of the block); warps 8-11 drain
-// dQ^T (thread = one of the CTA's 128 head-dim columns); warp 12 issues the
+// dQ^T (thread = one of the CTA's 128 head-dim columns) through a staging
+// buffer, 16 query rows at a time, each chunk added to the CTA's half of the
+// dQacc rows by one 2-D tensor bulk reduction; warp 12 issues the
 // MMAs; warp 13 issues the TMA loads.  Every wait is bounded.
 #pragma once
 
@@ -52,7 +54,10 @@ struct Bwd256Cfg {
   static constexpr int OFF_Q_OWN = 2 * KV_TILE, OFF_Q_OTH = OFF_Q_OWN + HALF;
   static constexpr int OFF_DO_OWN = OFF_Q_OTH + HALF, OFF_DO_OTH = OFF_DO_OWN + HALF;
   static constexpr int OFF_DS = OFF_DO_OTH + HALF;            // dS, [key][query]: one 128-row region
-  static constexpr int OFF_VEC = OFF_DS + KREG;               // lse2[BM] then D[BM]
+  static constexpr int CHUNK_ROWS = 16;                       // query rows per dQ reduction (tm_dq's box)
+  static constexpr int OFF_STG = OFF_DS + KREG;               // two dQ chunks, [row][owned d] fp32
+  static constexpr int STG_BYTES = 2 * CHUNK_ROWS * DH * 4;
+  static constexpr int OFF_VEC = OFF_STG + STG_BYTES;         // lse2[BM] then D[BM]
   static constexpr int VEC_BYTES = 2 * BM * 4;
   static constexpr int OFF_BAR = OFF_VEC + VEC_BYTES;
   static constexpr int N_BARS = 20;
@@ -82,7 +87,7 @@ template <bool PACKED>
 __global__ void __launch_bounds__(Bwd256Cfg::THREADS, 1)
 fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                 const BwdArgs args) {
+                 const __grid_constant__ CUtensorMap tm_dq, const BwdArgs args) {
   using C = Bwd256Cfg;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   int bh, kb, own;
@@ -426,14 +431,22 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else {
     // ------------------------------------------------------------ dQ drain (thread = owned head-dim column)
+    // Chunks of 16 query rows go row-major ([row][owned d], fp32) into one of two
+    // staging buffers and one thread adds each to dQacc with a tensor bulk
+    // reduction of the map's 128 x 16 box.  Rows past the sequence end are
+    // included (their dS, so their dQ, is exactly zero: P = 2^-inf there) and
+    // rows past the accumulator are not written.  The wait for each block ends
+    // in a vote of the four drain warps, so none is left at a named barrier.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
     const int dl = (warp - 8) * 32 + lane;
+    const bool issuer = dl == 0;
     const uint32_t tDQ = tmem + (static_cast<uint32_t>((warp - 8) * 32) << 16) + C::T_DQ;
+    float* stg = reinterpret_cast<float*>(smem + C::OFF_STG);
+    int last_buf = 1;                                  // staging buffer of the newest reduction
     for (int it = 0; it < n_iter; ++it) {
-      if (!mbar_wait_warp(b_dq_full, static_cast<uint32_t>(it) & 1u, ctl)) break;
+      if (!named_bar_and(1, C::DRAIN_THREADS, mbar_wait_warp(b_dq_full, static_cast<uint32_t>(it) & 1u, ctl))) break;
       tc_fence_after();
       const int q0 = q_row0(it);
-      float* acc = args.dq_acc + row_index<PACKED>(args.L, sp, q_head(it), q0) * C::D + col0 + dl;
       const int nq = min(C::BM, sp.nq - q0);
       uint32_t r[64];
       tmem_ld32(tDQ, *reinterpret_cast<uint32_t(*)[32]>(r));
@@ -443,15 +456,31 @@ fa_bwd256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(r + 32));
       tc_fence_before();
       mbar_arrive(b_dq_free);
-      if (nq >= C::BM) {
 #pragma unroll
-        for (int c = 0; c < C::BM; ++c) red_add_f32(acc + static_cast<size_t>(c) * C::D, __uint_as_float(r[c]));
-      } else {
+      for (int c = 0; c < C::BM / C::CHUNK_ROWS; ++c) {   // chunk c: queries 16c .. 16c + 15 of the block
+        if (C::CHUNK_ROWS * c >= nq) break;               // uniform over the drain warps
+        // the reduction that used this buffer before has read it: the newest one
+        // when a ragged block ended on this buffer, else the one before it
+        if (issuer) {
+          if ((c & 1) == last_buf) bulk_wait_read<0>();
+          else bulk_wait_read<1>();
+        }
+        last_buf = c & 1;
+        named_bar_sync(1, C::DRAIN_THREADS);
+        float* buf = stg + (c & 1) * C::CHUNK_ROWS * C::DH;
 #pragma unroll
-        for (int c = 0; c < C::BM; ++c)
-          if (c < nq) red_add_f32(acc + static_cast<size_t>(c) * C::D, __uint_as_float(r[c]));
+        for (int j = 0; j < C::CHUNK_ROWS; ++j) buf[j * C::DH + dl] = __uint_as_float(r[C::CHUNK_ROWS * c + j]);
+        fence_proxy_async_smem();
+        named_bar_sync(1, C::DRAIN_THREADS);
+        if (issuer) {
+          const long long row = row_index<PACKED>(args.L, sp, q_head(it), q0 + C::CHUNK_ROWS * c);
+          tma_reduce_add_2d(&tm_dq, sbase + C::OFF_STG + (c & 1) * C::CHUNK_ROWS * C::DH * 4, col0,
+                            static_cast<int>(row));
+          bulk_commit();
+        }
       }
     }
+    if (issuer) bulk_wait_all();
   }
 
   tc_fence_before();

@@ -144,6 +144,21 @@ bool make_map4(CUtensorMap* m, const void* base, int d, int rows, int heads, int
   return r == CUDA_SUCCESS;
 }
 
+// 2-D map of the fp32 dQ accumulator at head dim 256, [rows][256], for the
+// backward's tensor bulk reductions: box of 128 columns (one CTA's half of d) by
+// `box_rows` rows, no swizzle.
+bool make_map_dq256(CUtensorMap* m, float* acc, long long rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(rows < 1 ? 1 : rows)};
+  cuuint64_t strides[1] = {256 * 4};
+  cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, acc, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 fa_strides dense_strides(int H, int N, int d) {
   fa_strides st;
   st.row = d;
@@ -629,12 +644,14 @@ fa_status bwd_impl(int phases, const void* q, const void* k, const void* v, cons
     const long long grid = static_cast<long long>(a.n_kb) * a.bh_kv * (d == 256 ? 2 : 1);
     if (grid >= (1LL << 31)) return FA_ERR_INVALID;
     if (d == 256) {
+      CUtensorMap tdq;
+      if (!make_map_dq256(&tdq, a.dq_acc, a.acc_rows, Bwd256Cfg::CHUNK_ROWS)) return FA_ERR_CUDA;
       if (pk)
         fa_bwd256_kernel<true><<<static_cast<unsigned>(grid), Bwd256Cfg::THREADS, Bwd256Cfg::SMEM_BYTES, stream>>>(
-            tq, tk, tv, tdo, a);
+            tq, tk, tv, tdo, tdq, a);
       else
         fa_bwd256_kernel<false><<<static_cast<unsigned>(grid), Bwd256Cfg::THREADS, Bwd256Cfg::SMEM_BYTES, stream>>>(
-            tq, tk, tv, tdo, a);
+            tq, tk, tv, tdo, tdq, a);
     } else if (d == 64)
       launch_bwd_main<64>(pk, static_cast<unsigned>(grid), tq, tk, tv, tdo, a, stream);
     else
