@@ -208,7 +208,10 @@ struct BwdCfg {
   // (four warps share a sub-partition's 16K registers); P/dS warps take 144,
   // the MMA and TMA warps 112, the drain warps give theirs down to 80:
   // 256 * 144 + 128 * 80 + 64 * 112 = 54272 <= 448 * 128, and per sub-partition
-  // 2 * 144 + 80 + 112 = 480 <= 512 registers per thread slot.
+  // 2 * 144 + 80 + 112 = 480 <= 512 registers per thread slot.  setmaxnreg.inc
+  // draws on registers freed in its own sub-partition, so each must free what its
+  // warps take: sub-partitions 2 and 3 hold two P/dS warps (+16 each) and one
+  // drain warp (-48); a split that does not balance there waits forever.
   static constexpr int LAUNCH_REGS = 128;
   static constexpr int REGS_PDS = 144, REGS_DRAIN = 80, REGS_SINGLE = 112;
   static constexpr int REG = 128 * 128;        // one 64-column SW128 region of a 128-row bf16 tile
@@ -247,6 +250,9 @@ static_assert(BwdCfg<128>::PDS_THREADS * BwdCfg<128>::REGS_PDS + BwdCfg<128>::DR
               "register split exceeds the registers the block launches with");
 static_assert(2 * BwdCfg<128>::REGS_PDS + BwdCfg<128>::REGS_DRAIN + BwdCfg<128>::REGS_SINGLE <= 512,
               "register split exceeds a sub-partition");
+static_assert(2 * (BwdCfg<128>::REGS_PDS - BwdCfg<128>::LAUNCH_REGS) <=
+                  BwdCfg<128>::LAUNCH_REGS - BwdCfg<128>::REGS_DRAIN,
+              "register split does not balance within a sub-partition");
 
 // Work item x -> (head, key block).  Heads are taken in groups of
 // heads_per_group; inside a group the key blocks with the most query blocks

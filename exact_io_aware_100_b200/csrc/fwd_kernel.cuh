@@ -66,7 +66,10 @@ struct FwdCfg {
   static constexpr int THREADS = 384;
   // Register split (setmaxnreg): 384 threads launch with 168 registers each
   // (three warps per sub-partition); the eight softmax warps take 224, the
-  // other four give theirs down to 56: 256 * 224 + 128 * 56 = 384 * 168.
+  // other four give theirs down to 56: 256 * 224 + 128 * 56 = 384 * 168.  It
+  // also balances within each sub-partition, where setmaxnreg.inc draws its
+  // registers from: two softmax warps take 2 * (224 - 168) = 112, which the one
+  // other warp there frees (168 - 56).
   static constexpr int LAUNCH_REGS = 168;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
