@@ -566,7 +566,7 @@ def run_varlen(args, w, fa, torch, dist, world, rank, local_rank, dev):
 # before every step whose inputs and outputs fit in twice the L2), one after the other in the same
 # process.
 CONFIG_TABLE = (("1", "single_head", 20), ("2", "multi_head", 20), ("2c", "multi_head_causal", 20),
-                ("4", "long_context", 3), ("5", "backward", 10))
+                ("3nc", "prefill_noncausal", 5), ("4", "long_context", 3), ("5", "backward", 10))
 
 
 def _device_inputs(torch, dev, w, names, seed):

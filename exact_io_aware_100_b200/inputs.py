@@ -11,6 +11,7 @@ or 128, causal and non-causal, long sequences):
   ``single_head``  B=1  H=1  N=128    d=64   fp32 inputs, non-causal
   ``multi_head``   B=4  H=16 N=2048   d=64   bf16, non-causal and causal
   ``prefill``      B=2  H=32 N=8192   d=128  bf16, K scaled by 2, causal
+  ``prefill_noncausal``  the same, non-causal
   ``long_context`` B=1  H=16 N=65536  d=128  bf16, causal
   ``backward``     B=4  H=16 N=4096   d=128  bf16 Q,K,V,dO, causal
 
@@ -78,6 +79,7 @@ WORKLOADS = {
     "multi_head": Workload("multi_head", 4, 16, 2048, 64, False, "bf16", 1.0, 1002),
     "multi_head_causal": Workload("multi_head_causal", 4, 16, 2048, 64, True, "bf16", 1.0, 1002),
     "prefill": Workload("prefill", 2, 32, 8192, 128, True, "bf16", 2.0, 1003),
+    "prefill_noncausal": Workload("prefill_noncausal", 2, 32, 8192, 128, False, "bf16", 2.0, 1010),
     "long_context": Workload("long_context", 1, 16, 65536, 128, True, "bf16", 1.0, 1004),
     "backward": Workload("backward", 4, 16, 4096, 128, True, "bf16", 1.0, 1005, True),
     # grouped-query attention on the prefill shape: 32 query heads over 8 key/value heads

@@ -82,6 +82,27 @@ def test_prefill_backward_full_size_sampled_heads():
         assert np.isfinite(to_f64(x)).all()
 
 
+def test_prefill_noncausal_full_size():
+    """The prefill shape without the causal mask (B=2 H=32 N=8192 d=128, K x2), as the benchmark's
+    configuration table times it: the forward on sampled rows of heads from different tile groups,
+    the backward on two whole heads."""
+    import exact_io_aware_100_b200 as fa
+    w = inputs.WORKLOADS["prefill_noncausal"]
+    host = inputs.make_inputs(w, names=("q", "k", "v", "do"))
+    t = _bf16(host)
+    o, lse = fa.forward(t["q"], t["k"], t["v"], w.causal)
+    dq, dk, dv = fa.backward(t["q"], t["k"], t["v"], o, lse, t["do"], w.causal)
+    _status_ok()
+    _sampled_rows(w, host, o, lse, (0, 21, 42, 63), rows_per_head=128)
+    for bh in (5, 50):
+        b, h = divmod(bh, w.H)
+        f = {n: inputs.to_f64(host[n][b:b + 1, h:h + 1], "bf16") for n in ("q", "k", "v", "do")}
+        ref = attention_bwd(f["q"], f["k"], f["v"], f["do"], w.scale, w.causal)
+        bound = bwd_operand_rounding_bound(f["q"], f["k"], f["v"], f["do"], w.scale, w.causal)
+        for name, got, rr, bb in zip(("dq", "dk", "dv"), (dq, dk, dv), ref, bound):
+            assert_close_bwd(name, to_f64(got[b, h]), rr[0, 0], bb[0, 0])
+
+
 def test_prefill_gqa_full_size():
     """32 query heads over 8 key/value heads at the prefill sizes: forward rows from both causal
     tile groups, and the backward of whole key/value heads (each the sum over its four query
