@@ -49,6 +49,15 @@ def test_single_head_fp32_inputs():
     assert ma < 3e-2 and rl < 1e-2, (ma, rl)
 
 
+@pytest.mark.parametrize("B,H,N,d,causal", [
+    (1, 1, 1, 64, True), (2, 3, 17, 64, False), (1, 2, 100, 128, True), (2, 2, 128, 128, False),
+    (1, 1, 128, 64, True), (1, 2, 129, 64, True), (1, 1, 300, 128, False),
+])
+def test_fp32_inputs_short_and_long(B, H, N, d, causal):
+    """fa_fwd_ex(FA_F32) on short and ragged lengths: cast to bf16, then the tensor-core kernel."""
+    full_check(B, H, N, d, causal, 8800 + N + d, dtype="f32")
+
+
 @pytest.mark.parametrize("name", ["multi_head", "multi_head_causal"])
 def test_multi_head(name):
     w = inputs.WORKLOADS[name]
