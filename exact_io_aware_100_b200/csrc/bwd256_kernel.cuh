@@ -75,6 +75,10 @@ static_assert(Bwd256Cfg::T_P + 32 <= Bwd256Cfg::TMEM_COLS, "tensor memory plan")
 static_assert(Bwd256Cfg::PDS_THREADS * 144 + Bwd256Cfg::DRAIN_THREADS * 80 + 64 * 112 <=
                   Bwd256Cfg::THREADS * Bwd256Cfg::LAUNCH_REGS,
               "register split exceeds the registers the block launches with");
+// setmaxnreg.inc takes registers freed in its own sub-partition: in sub-partitions
+// 2 and 3 two P/dS warps (+16 each) against one drain warp (-48)
+static_assert(2 * (144 - Bwd256Cfg::LAUNCH_REGS) <= Bwd256Cfg::LAUNCH_REGS - 80,
+              "register split does not balance within a sub-partition");
 
 // Work item x -> (key/value head bh, key block kb, owned half c).  The two halves
 // of a key block are neighbours, so they read the same K, V, Q and dO from L2.

@@ -43,6 +43,8 @@ struct FwdSpCfg {
   // Register split as in fwd_kernel.cuh: 384 threads launch with 168 registers;
   // the eight softmax warps take 224, the other four give theirs down to 56.
   static constexpr int LAUNCH_REGS = 168;
+  static_assert(2 * (224 - LAUNCH_REGS) <= LAUNCH_REGS - 56,
+                "register split does not balance within a sub-partition");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_O0 = 0, T_O1 = D, T_S0 = 2 * D, T_S1 = 2 * D + BN, T_P0 = 2 * D + 2 * BN,
                             T_P1 = 2 * D + 2 * BN + BN / 2;

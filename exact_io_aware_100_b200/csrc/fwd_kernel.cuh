@@ -71,6 +71,8 @@ struct FwdCfg {
   // registers from: two softmax warps take 2 * (224 - 168) = 112, which the one
   // other warp there frees (168 - 56).
   static constexpr int LAUNCH_REGS = 168;
+  static_assert(2 * (224 - LAUNCH_REGS) <= LAUNCH_REGS - 56,
+                "register split does not balance within a sub-partition");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
   // shared-memory layout (offsets from a 1024-aligned base)
